@@ -1,0 +1,238 @@
+"""Seeded synthetic inputs for Hybrid Tree Attention verification calls.
+
+This module draws the random tensors and tree shapes that both the CUDA path
+and the CPU oracle consume.  It holds none of the attention arithmetic: only
+random draws, rounding to bf16 and the tree topology.
+
+Recipe (every workload):
+  * One ``torch.Generator('cpu')`` per (seed, stream, b, head), seeded from
+    ``numpy.random.SeedSequence([seed, stream, b, head])``.  So one head's
+    K/V can be regenerated alone (sampled parity at full size), and the bytes
+    do not depend on the device.
+  * Q, K, V drawn N(0, 1) in fp32 and rounded to bf16 (round to nearest even,
+    by torch).  In "peaked" workloads each K row (prefix and tree keys alike)
+    is multiplied in fp32 by one scalar 1 + |N(0, 1)| before the rounding.
+  * Trees: "levels" -- node ids in breadth-first level order, level widths
+    ``widths`` (4 16 16 16 16 -> 68 nodes, the ``--tree_shape`` of the LongSpec
+    README's evaluation commands); level-1 nodes hang off the prefix end
+    (parent -1) and each deeper node's parent is uniform over the previous
+    level's ids.  "random" -- node 0 has parent -1, node i >= 1 a parent
+    uniform over 0..i-1.  "chain" -- parent[i] = i - 1.
+  * Prefix lengths: fixed L, or uniform integers in [lo, hi] per sequence.
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+# stream ids of the random draws
+_S_Q, _S_KP, _S_VP, _S_KT, _S_VT, _S_KSCALE, _S_TREE, _S_LEN = range(8)
+
+LONGSPEC_TREE_SHAPE = (4, 16, 16, 16, 16)
+
+
+def _generator(seed: int, stream: int, b: int = 0, h: int = 0) -> torch.Generator:
+    state = np.random.SeedSequence([int(seed), int(stream), int(b), int(h)])
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(state.generate_state(1, dtype=np.uint64)[0] & ((1 << 63) - 1)))
+    return g
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> numpy uint16 bit patterns (no copy of values' meaning)."""
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected a bf16 tensor")
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def tree_levels(widths, g: torch.Generator) -> np.ndarray:
+    parent = []
+    prev = []
+    nid = 0
+    for lvl, w in enumerate(widths):
+        cur = list(range(nid, nid + w))
+        for _ in cur:
+            if lvl == 0:
+                parent.append(-1)
+            else:
+                k = int(torch.randint(len(prev), (1,), generator=g).item())
+                parent.append(prev[k])
+        prev = cur
+        nid += w
+    return np.asarray(parent, dtype=np.int32)
+
+
+def tree_random(T: int, g: torch.Generator) -> np.ndarray:
+    parent = [-1] if T > 0 else []
+    for i in range(1, T):
+        parent.append(int(torch.randint(i, (1,), generator=g).item()))
+    return np.asarray(parent, dtype=np.int32)
+
+
+def tree_chain(T: int) -> np.ndarray:
+    return np.arange(-1, T - 1, dtype=np.int32)
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shapes and seed of one verification-attention call.
+
+    q [B][Hq][T][D], k/v_prefix [B][Hkv][L_cap][D], k/v_tree [B][Hkv][T][D],
+    prefix_len [B], parent [B][T]; bf16 tensors, int32 index arrays.
+    """
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    T: int
+    L_cap: int
+    seed: int
+    tree: str = "levels"                      # levels | random | chain
+    widths: Tuple[int, ...] = LONGSPEC_TREE_SHAPE
+    prefix_range: Optional[Tuple[int, int]] = None   # None -> every L_b = L_cap
+    k_peaked: bool = False
+    scale: float = 0.0                        # 0 -> 1/sqrt(D)
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+    # ---- index inputs -------------------------------------------------
+    def prefix_lens(self) -> np.ndarray:
+        if self.prefix_range is None:
+            return np.full((self.B,), self.L_cap, dtype=np.int32)
+        lo, hi = self.prefix_range
+        g = _generator(self.seed, _S_LEN)
+        return torch.randint(lo, hi + 1, (self.B,), generator=g).to(torch.int32).numpy()
+
+    def parents(self) -> np.ndarray:
+        out = np.zeros((self.B, self.T), dtype=np.int32)
+        for b in range(self.B):
+            g = _generator(self.seed, _S_TREE, b)
+            if self.tree == "levels":
+                if sum(self.widths) != self.T:
+                    raise ValueError("level widths do not add up to T")
+                out[b] = tree_levels(self.widths, g)
+            elif self.tree == "random":
+                out[b] = tree_random(self.T, g)
+            elif self.tree == "chain":
+                out[b] = tree_chain(self.T)
+            else:
+                raise ValueError(f"unknown tree kind {self.tree}")
+        return out
+
+    # ---- per-head random tensors ------------------------------------------
+    def _key_scale(self, b: int, kvh: int) -> torch.Tensor:
+        g = _generator(self.seed, _S_KSCALE, b, kvh)
+        return 1.0 + torch.randn(self.L_cap + self.T, generator=g).abs()
+
+    def q_head(self, b: int, h: int) -> torch.Tensor:
+        g = _generator(self.seed, _S_Q, b, h)
+        return torch.randn(self.T, self.D, generator=g).to(torch.bfloat16)
+
+    def k_prefix_head(self, b: int, kvh: int) -> torch.Tensor:
+        g = _generator(self.seed, _S_KP, b, kvh)
+        k = torch.randn(self.L_cap, self.D, generator=g)
+        if self.k_peaked:
+            k *= self._key_scale(b, kvh)[: self.L_cap, None]
+        return k.to(torch.bfloat16)
+
+    def v_prefix_head(self, b: int, kvh: int) -> torch.Tensor:
+        g = _generator(self.seed, _S_VP, b, kvh)
+        return torch.randn(self.L_cap, self.D, generator=g).to(torch.bfloat16)
+
+    def k_tree_head(self, b: int, kvh: int) -> torch.Tensor:
+        g = _generator(self.seed, _S_KT, b, kvh)
+        k = torch.randn(self.T, self.D, generator=g)
+        if self.k_peaked:
+            k *= self._key_scale(b, kvh)[self.L_cap:, None]
+        return k.to(torch.bfloat16)
+
+    def v_tree_head(self, b: int, kvh: int) -> torch.Tensor:
+        g = _generator(self.seed, _S_VT, b, kvh)
+        return torch.randn(self.T, self.D, generator=g).to(torch.bfloat16)
+
+    # ---- whole tensors ------------------------------------------------
+    def generate(self, with_prefix: bool = True) -> dict:
+        """All inputs as CPU tensors (bf16 / int32)."""
+        B, Hq, Hkv, D, T, L = self.B, self.Hq, self.Hkv, self.D, self.T, self.L_cap
+        q = torch.empty(B, Hq, T, D, dtype=torch.bfloat16)
+        kt = torch.empty(B, Hkv, T, D, dtype=torch.bfloat16)
+        vt = torch.empty(B, Hkv, T, D, dtype=torch.bfloat16)
+        for b in range(B):
+            for h in range(Hq):
+                q[b, h] = self.q_head(b, h)
+            for h in range(Hkv):
+                kt[b, h] = self.k_tree_head(b, h)
+                vt[b, h] = self.v_tree_head(b, h)
+        out = dict(q=q, k_tree=kt, v_tree=vt,
+                   prefix_len=torch.from_numpy(self.prefix_lens()),
+                   parent=torch.from_numpy(self.parents()))
+        if with_prefix:
+            kp = torch.empty(B, Hkv, L, D, dtype=torch.bfloat16)
+            vp = torch.empty(B, Hkv, L, D, dtype=torch.bfloat16)
+            for b in range(B):
+                for h in range(Hkv):
+                    kp[b, h] = self.k_prefix_head(b, h)
+                    vp[b, h] = self.v_prefix_head(b, h)
+            out["k_prefix"] = kp
+            out["v_prefix"] = vp
+        return out
+
+    def generate_head(self, b: int, kvh: int) -> dict:
+        """Inputs restricted to one (b, KV head): the G query heads of that
+        group and that head's prefix/tree K, V, as a B=1, Hkv=1 problem."""
+        G = self.Hq // self.Hkv
+        q = torch.stack([self.q_head(b, kvh * G + g) for g in range(G)])[None]
+        return dict(
+            q=q,
+            k_prefix=self.k_prefix_head(b, kvh)[None, None],
+            v_prefix=self.v_prefix_head(b, kvh)[None, None],
+            k_tree=self.k_tree_head(b, kvh)[None, None],
+            v_tree=self.v_tree_head(b, kvh)[None, None],
+            prefix_len=torch.from_numpy(self.prefix_lens()[b:b + 1].copy()),
+            parent=torch.from_numpy(self.parents()[b:b + 1].copy()),
+        )
+
+    # ---- sizes ------------------------------------------------------------
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    def algorithmic_bytes(self) -> int:
+        """Bytes one call must move at minimum: prefix K+V of the L_b keys
+        actually present, Q, tree K+V, out (bf16), lse (fp32), parent and
+        prefix_len (int32)."""
+        lens = self.prefix_lens().astype(np.int64)
+        kv = int(2 * self.Hkv * self.D * 2 * lens.sum())
+        q = self.B * self.Hq * self.T * self.D * 2
+        tree = 2 * self.B * self.Hkv * self.T * self.D * 2
+        out = self.B * self.Hq * self.T * self.D * 2
+        lse = self.B * self.Hq * self.T * 4
+        idx = self.B * self.T * 4 + self.B * 4
+        return kv + q + tree + out + lse + idx
+
+
+# The attention shapes of the models the LongSpec pages evaluate, with the
+# pages' 4/16/16/16/16 draft tree.  The datasets of the pages (LongBench,
+# RepoBench-P, AIME24, MATH500) are not used: these draws stand in for them.
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, Hq=2, Hkv=1, D=64, T=8, L_cap=256, seed=0,
+                     tree="random"),
+    "llama3-8b-32k": Workload("llama3-8b-32k", B=1, Hq=32, Hkv=8, D=128,
+                              T=68, L_cap=32768, seed=1),
+    "vicuna-7b-b8": Workload("vicuna-7b-b8", B=8, Hq=32, Hkv=32, D=128, T=68,
+                             L_cap=16384, seed=2, prefix_range=(8192, 16384)),
+    "qwq-32b-32k-peaked": Workload("qwq-32b-32k-peaked", B=1, Hq=40, Hkv=8,
+                                   D=128, T=68, L_cap=32768, seed=3,
+                                   k_peaked=True),
+    "ultra-256k": Workload("ultra-256k", B=1, Hq=32, Hkv=8, D=128, T=68,
+                           L_cap=262144, seed=4),
+    "ultra-256k-chain5": Workload("ultra-256k-chain5", B=1, Hq=32, Hkv=8,
+                                  D=128, T=5, L_cap=262144, seed=5,
+                                  tree="chain"),
+}
