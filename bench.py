@@ -1,0 +1,371 @@
+"""Benchmark of one Hybrid Tree Attention verification call (one layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--num-splits S]
+
+A step is one full verification call (prefix split-KV kernel, then the tree
+pass fused with the log-sum-exp merge) over one batch of synthetic inputs
+already resident in HBM.  Inputs rotate over enough buffer sets that every
+step's K/V are not in L2 (126 MB) when it starts.  The metric is the
+microseconds per layer call (lower is better) and, for the prefix kernel,
+the achieved HBM bandwidth against the measured peak.
+
+Under torchrun (N > 1) every rank runs its own calls on its own GPU (weak
+scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from tree_masked_verification_b200 import hta  # noqa: E402
+from tree_masked_verification_b200.inputs import WORKLOADS  # noqa: E402
+
+METRIC = "µs per layer verify-attention call; achieved HBM GB/s vs B200 peak @32k prefix"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(w, S, n_sets):
+    tree = {"levels": "/".join(map(str, w.widths)), "random": "random", "chain": "chain"}[w.tree]
+    lens = w.prefix_lens()
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "T": w.T,
+            "L_cap": w.L_cap, "L_mean": float(lens.mean()), "tree": tree,
+            "k_peaked": w.k_peaked, "num_splits": S,
+            "l2": f"inputs rotate over {n_sets} buffer sets ({n_sets}x the K/V bytes > 2x L2)"
+            if n_sets > 1 else "K/V bytes per call > 2x L2"}
+
+
+def prefix_algorithmic_bytes(w):
+    """Bytes the prefix kernel must move at minimum: K and V of the L_b
+    prefix keys of every (b, KV head) (2 * D * 2 bytes per key and head),
+    plus Q once.  The split partials are not counted."""
+    lens = w.prefix_lens().astype(np.int64)
+    return int(lens.sum()) * w.Hkv * 2 * w.D * 2 + w.B * w.Hq * w.T * w.D * 2
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# --------------------------------------------------------------------------
+# CPU oracle: the reported baseline (cpu_baseline) and the reference arm
+# --------------------------------------------------------------------------
+_ORACLE_CACHE = {}
+
+
+def _oracle_head_problem(w, b, kvh):
+    """The oracle problem of one (b, KV head) group (B = 1, Hkv = 1)."""
+    import oracle
+    from tree_masked_verification_b200.inputs import bf16_bits
+    key = (w.name, b, kvh)
+    if key not in _ORACLE_CACHE:
+        inp = w.generate_head(b, kvh)
+        _ORACLE_CACHE.clear()
+        _ORACLE_CACHE[key] = oracle.Problem(
+            bf16_bits(inp["q"]), bf16_bits(inp["k_prefix"]), bf16_bits(inp["v_prefix"]),
+            inp["prefix_len"].numpy(), bf16_bits(inp["k_tree"]), bf16_bits(inp["v_tree"]),
+            inp["parent"].numpy(), scale=w.scale)
+    return _ORACLE_CACHE[key]
+
+
+def oracle_rows_timed(w, heads, budget_s, rows_per_head=None, row_offset=0):
+    """Runs the fp64 oracle (single thread) over the packed rows of the given
+    (b, KV head) groups until `budget_s` is spent; returns (seconds, rows).
+    Input generation is outside the timed part."""
+    done, spent = 0, 0.0
+    M = w.G * w.T
+    for b, kvh in heads:
+        p = _oracle_head_problem(w, b, kvh)
+        n = M if rows_per_head is None else min(M, rows_per_head)
+        rows = np.array([[0, ((row_offset + r) % M) // w.T, ((row_offset + r) % M) % w.T]
+                         for r in range(n)], dtype=np.int32)
+        t0 = time.perf_counter()
+        p.attention(rows)
+        spent += time.perf_counter() - t0
+        done += n
+        if spent >= budget_s:
+            break
+    return spent, done
+
+
+def cpu_baseline(w, budget_s=10.0):
+    heads = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    spent, rows = oracle_rows_timed(w, heads, budget_s)
+    total_rows = w.B * w.Hq * w.T
+    us_per_call = spent / rows * total_rows * 1e6
+    return {"value": us_per_call, "unit": "µs", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of {total_rows} query rows (whole KV-head groups, fp64, one "
+                      f"thread, {spent:.1f} s), scaled to one full call"}
+
+
+def run_reference(args, world, rank):
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    total_rows = w.B * w.Hq * w.T
+    per_step = max(1, min(w.G * w.T, args.ref_rows))
+    heads = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    times = []
+    for i in range(args.warmup + args.steps):
+        spent, rows = oracle_rows_timed(w, heads[:1], 0.0, rows_per_head=per_step,
+                                        row_offset=i * per_step)
+        if i >= args.warmup:
+            times.append(spent / rows)
+    sec_per_row = sum(times) / len(times)
+    us = sec_per_row * total_rows * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "µs",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec_per_row * per_step * 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, None, 1),
+        "cpu_baseline": {"value": us, "unit": "µs", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} query rows per step of {total_rows}, fp64, "
+                                   f"one thread, scaled to one full call"},
+        "e2e": {"value": us, "unit": "µs", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cpu = w.generate()
+    kv_bytes = 2 * cpu["k_prefix"].numel() * 2
+    n_sets = 1 if kv_bytes > 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / kv_bytes)) + 1
+    sets = []
+    base = {k: v.to(dev) for k, v in cpu.items()}
+    for i in range(n_sets):
+        sets.append(base if i == 0 else {k: v.clone() for k, v in base.items()})
+    dims = hta.dims_of(base["q"], base["k_prefix"], w.scale)
+    S, chunk = hta.chunking(dims, args.num_splits)
+    ws = hta.new_workspace(dims, args.num_splits, dev)
+    out = torch.empty_like(base["q"])
+    lse = torch.empty(base["q"].shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(i, events=None):
+        s = sets[i % n_sets]
+        hta.verify(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], s["k_tree"],
+                   s["v_tree"], s["parent"], out=out, lse=lse, workspace=ws, scale=w.scale,
+                   num_splits=args.num_splits, prefix_events=events, stream=stream)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    if hta.get_status(ws) != hta.OK:
+        raise RuntimeError("device status error during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local if world > 1 else 0)
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        call(i, ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    prefix_ms = [a.elapsed_time(b) for a, b in ev]
+    prefix_avg_ms = max_over_ranks(sum(prefix_ms) / len(prefix_ms), world)
+    if hta.get_status(ws) != hta.OK:
+        raise RuntimeError("device status error in the timed region")
+
+    ms_per_step = elapsed_ms / args.steps
+    us_per_call = ms_per_step * 1e3 / world
+    peak, peak_kind = peaks()
+    pbytes = prefix_algorithmic_bytes(w)
+    achieved = pbytes / (prefix_avg_ms * 1e-3) / 1e9
+    call_bytes = w.algorithmic_bytes()
+
+    # end to end through the host-buffer entry point (copies inside the region)
+    e2e = run_e2e(args, w, cpu, dims, dev, stream, world)
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": us_per_call, "unit": "µs", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, 4/16/16/16/16 tree)",
+        "config": workload_config(w, S, n_sets),
+        "roofline": {"bound": "hbm", "kernel": "prefix_tc_kernel", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes": pbytes, "avg_launch_us": prefix_avg_ms * 1e3},
+        "call_roofline": {"bytes": call_bytes, "achieved_gbs": call_bytes / (ms_per_step * 1e-3) / 1e9,
+                          "frac_measured": call_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
+                          "frac_nominal_8tbs": call_bytes / (ms_per_step * 1e-3) / 8e12},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, cpu, dims, dev, stream, world):
+    host = {k: v.pin_memory() for k, v in cpu.items()}
+    arena = torch.empty(hta.host_arena_bytes(dims), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(host["q"]).pin_memory()
+    lse = torch.empty(host["q"].shape[:3], dtype=torch.float32).pin_memory()
+
+    def call():
+        hta.verify_host(host["q"], host["k_prefix"], host["v_prefix"], host["prefix_len"],
+                        host["k_tree"], host["v_tree"], host["parent"], out, lse, arena,
+                        scale=w.scale, stream=stream)
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(min(args.warmup, 3)):
+        call()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    return {"value": ms * 1e3 / world, "unit": "µs", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3-8b-32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

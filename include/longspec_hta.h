@@ -1,0 +1,229 @@
+/*
+ * longspec_hta.h -- C ABI of Hybrid Tree Attention on B200 (sm_100a).
+ *
+ * Hybrid Tree Attention is the verification attention of LongSpec's
+ * long-context speculative decoding.  For every query head, T speculated
+ * tree tokens attend
+ *   - to the long shared prefix KV cache, with no mask, and
+ *   - to each other, under the tree mask: a token sees itself and its
+ *     ancestors (parent[] chain up to -1, which stands for the prefix end).
+ * The prefix part and the tree part are computed as two softmax partials and
+ * merged exactly by log-sum-exp rescaling.
+ *
+ * Passages that define the operation:
+ *   - LongSpec README (sail-sg/LongSpec), "Introduction", contribution
+ *     "Hybrid Attention Aggregation": fast prefix computation combined with
+ *     standard attention for tree mask handling.
+ *   - LongSpec paper summary (Elamur Research), "Summary", Hybrid Tree
+ *     Attention bullet: verification split into a Flash Attention pass over
+ *     the prefix and a kernel for the speculated tree; "Key points": target
+ *     attention latency 49.92 ms -> 12.54 ms (hardware not given).
+ *   - LongSpec arXiv abstract (original English abstract): attention
+ *     aggregation combining fast prefix implementations with standard
+ *     attention for tree mask handling; lossless (title).
+ *   - SpecExtend abstract (codewithpapers.app): Hybrid Tree Attention used as
+ *     a drop-in attention component.
+ *
+ * Conventions shared by every entry point
+ *   Layouts (row-major, no padding, all little-endian):
+ *     q          bf16  [B][Hq][T][D]
+ *     k_prefix   bf16  [B][Hkv][L_cap][D]     key j of sequence b valid for j < L_b
+ *     v_prefix   bf16  [B][Hkv][L_cap][D]
+ *     prefix_len int32 [B]                    0 <= L_b <= L_cap
+ *     k_tree     bf16  [B][Hkv][T][D]
+ *     v_tree     bf16  [B][Hkv][T][D]
+ *     parent     int32 [B][T]                 parent[i] in [-1, i); -1 = child of the prefix end
+ *     out        bf16  [B][Hq][T][D]
+ *     lse        fp32  [B][Hq][T]             natural log of sum exp(scale * q.k) over visible keys
+ *   Query head h reads KV head h / (Hq / Hkv) (contiguous GQA groups).
+ *   Device pointers unless stated; every pointer 16-byte aligned.
+ *   Ownership: the caller owns every buffer, the workspace included; the
+ *   library allocates no device memory in any call.
+ *   Streams: calls are asynchronous on `stream` (0 = legacy default stream);
+ *   only longspec_hta_get_status synchronises.
+ *   Return value: LONGSPEC_HTA_OK (0) or a negative longspec_hta_status.  A
+ *   call that returns an error launched nothing.  Problems only the device
+ *   can see (bad parent[], prefix_len out of range, a pipeline wait that ran
+ *   out) are recorded in the workspace status word, reported by
+ *   longspec_hta_get_status; the affected rows of `out`/`lse` are NaN.
+ *   Limits: D in {64, 128}; 1 <= T <= LONGSPEC_HTA_T_MAX; Hq % Hkv == 0;
+ *   B*Hq*T rows and B*Hkv*L_cap keys below 2^31.  No CPU fallback: on a
+ *   device other than sm_100 the calls return LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE.
+ */
+#ifndef LONGSPEC_HTA_H
+#define LONGSPEC_HTA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LONGSPEC_HTA_API __attribute__((visibility("default")))
+#else
+#define LONGSPEC_HTA_API
+#endif
+
+#define LONGSPEC_HTA_T_MAX 256
+#define LONGSPEC_HTA_ABI_VERSION 1
+
+typedef enum {
+    LONGSPEC_HTA_OK = 0,
+    LONGSPEC_HTA_ERR_INVALID_DIMS = -1,        /* sizes out of range, Hq % Hkv != 0, bad scale */
+    LONGSPEC_HTA_ERR_NULL_POINTER = -2,
+    LONGSPEC_HTA_ERR_MISALIGNED = -3,          /* a pointer not 16-byte aligned */
+    LONGSPEC_HTA_ERR_T_TOO_LARGE = -4,         /* T > LONGSPEC_HTA_T_MAX */
+    LONGSPEC_HTA_ERR_UNSUPPORTED_D = -5,       /* D not 64 or 128 */
+    LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL = -6,
+    LONGSPEC_HTA_ERR_CUDA = -7,                /* a CUDA runtime/driver call failed */
+    LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE = -8,  /* current device is not sm_100 */
+    LONGSPEC_HTA_ERR_INVALID_OPTION = -9,
+    /* device-detected, reported by longspec_hta_get_status */
+    LONGSPEC_HTA_ERR_BAD_PARENT = -16,         /* some parent[b][i] outside [-1, i) */
+    LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE = -17,   /* some prefix_len[b] outside [0, L_cap] */
+    LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT = -18    /* a bounded in-kernel wait ran out */
+} longspec_hta_status;
+
+/* Problem sizes of one call.  scale 0 means 1/sqrt(D); otherwise > 0. */
+typedef struct {
+    int B, Hq, Hkv, D, T, L_cap;
+    float scale;
+} longspec_hta_dims;
+
+/* Prefix kernels selectable through longspec_hta_options.prefix_kernel. */
+#define LONGSPEC_HTA_PREFIX_TCGEN05 0   /* TMA + tcgen05/TMEM split-KV kernel (default) */
+#define LONGSPEC_HTA_PREFIX_SIMT    1   /* plain CUDA-core split-KV kernel, for cross-checks */
+
+/* Optional knobs of longspec_hta_verify_ex.  Zero-initialise for defaults. */
+typedef struct {
+    int num_splits;          /* prefix split-KV chunks per (b, KV head); 0 = chosen by the library */
+    int prefix_kernel;       /* LONGSPEC_HTA_PREFIX_* */
+    cudaEvent_t prefix_begin;/* if non-null, recorded on `stream` right before the prefix kernel */
+    cudaEvent_t prefix_end;  /* if non-null, recorded on `stream` right after the prefix kernel */
+} longspec_hta_options;
+
+/* ABI version of the loaded library (LONGSPEC_HTA_ABI_VERSION). */
+LONGSPEC_HTA_API int longspec_hta_abi_version(void);
+
+/* Text of a status code; never NULL. */
+LONGSPEC_HTA_API const char *longspec_hta_strerror(int code);
+
+/* Split-KV chunk count the library uses for `dims` when num_splits = 0
+ * (number of SMs of the current device enters the choice).  Returns a
+ * negative status on invalid dims. */
+LONGSPEC_HTA_API int longspec_hta_default_splits(const longspec_hta_dims *dims);
+
+/* Split-KV chunking for a requested split count (0 = the default choice):
+ * writes the number of chunks S actually used and the chunk length in keys
+ * (a multiple of 128; chunk c covers prefix keys [c*C, (c+1)*C) clipped to
+ * [0, L_b)).  Either output may be NULL. */
+LONGSPEC_HTA_API int longspec_hta_chunking(const longspec_hta_dims *dims, int num_splits,
+                                           int *num_splits_out, int *chunk_keys_out);
+
+/* Workspace bytes needed by longspec_hta_verify(_ex) for `dims` and a split
+ * count (0 = the default choice).  Holds the status word and the fp32 prefix
+ * partials: B*Hq*T*S*(D+1)*4 bytes plus 256.  0 on invalid dims. */
+LONGSPEC_HTA_API size_t longspec_hta_workspace_bytes(const longspec_hta_dims *dims, int num_splits);
+
+/* Clears the workspace status word (asynchronously on `stream`).  Call once
+ * after allocating a workspace; longspec_hta_get_status clears it again. */
+LONGSPEC_HTA_API int longspec_hta_workspace_init(void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
+/*
+ * The verification attention of one layer: out and lse for every
+ * (b, h, t).  Runs the split-KV prefix kernel (TMA + tcgen05, accumulators
+ * in tensor memory) over prefix keys [0, L_b), then the tree kernel (ancestor
+ * bitmask built from parent[] in shared memory, masked online softmax over
+ * the tree keys) fused with the log-sum-exp merge of all partials.
+ * Two kernel launches on `stream`.
+ */
+LONGSPEC_HTA_API int longspec_hta_verify(const longspec_hta_dims *dims,
+                        const void *q, const void *k_prefix,
+                        const void *v_prefix, const int32_t *prefix_len,
+                        const void *k_tree, const void *v_tree,
+                        const int32_t *parent, void *out, float *lse,
+                        void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/* longspec_hta_verify with options (NULL = defaults). */
+LONGSPEC_HTA_API int longspec_hta_verify_ex(const longspec_hta_dims *dims,
+                           const void *q, const void *k_prefix,
+                           const void *v_prefix, const int32_t *prefix_len,
+                           const void *k_tree, const void *v_tree,
+                           const int32_t *parent, void *out, float *lse,
+                           void *workspace, size_t workspace_bytes,
+                           const longspec_hta_options *opts,
+                           cudaStream_t stream);
+
+/* Device bytes of the staging arena longspec_hta_verify_host needs: room
+ * for every input and output plus the workspace, each 256-byte aligned. */
+LONGSPEC_HTA_API size_t longspec_hta_host_arena_bytes(const longspec_hta_dims *dims);
+
+/*
+ * End-to-end call on HOST buffers (same layouts, host pointers; pinned
+ * memory gives asynchronous copies).  Copies the inputs into the caller's
+ * device `arena` (longspec_hta_host_arena_bytes), runs longspec_hta_verify,
+ * and copies out and lse back, all on `stream`; the host results are valid
+ * after the stream is synchronised.  The status word lives in the arena and
+ * is cleared by this call before the launch.
+ */
+LONGSPEC_HTA_API int longspec_hta_verify_host(const longspec_hta_dims *dims,
+                             const void *q, const void *k_prefix,
+                             const void *v_prefix, const int32_t *prefix_len,
+                             const void *k_tree, const void *v_tree,
+                             const int32_t *parent, void *out, float *lse,
+                             void *arena, size_t arena_bytes,
+                             cudaStream_t stream);
+
+/*
+ * Debug export of the tree mask: bits uint32 [B][T][ceil(T/32)], bit k of
+ * word w of row i set iff node 32w+k is node i or an ancestor of i.  Same
+ * device code as the tree kernel's shared-memory mask.  Bad parents are
+ * reported through the status word of `workspace` (>= 256 bytes) and their
+ * trees' rows are written as all ones.
+ */
+LONGSPEC_HTA_API int longspec_hta_tree_mask(const int32_t *parent, int B, int T, uint32_t *bits,
+                           void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/*
+ * Debug export of the tree partial alone: attention of every (b, h, t) over
+ * its visible tree keys only.  o_tree fp32 [B][Hq][T][D] (normalised),
+ * lse_tree fp32 [B][Hq][T] (natural log).  Same kernel as verify's tree pass.
+ * Needs a workspace of >= 256 bytes for the status word.
+ */
+LONGSPEC_HTA_API int longspec_hta_tree_partial(const longspec_hta_dims *dims, const void *q,
+                              const void *k_tree, const void *v_tree,
+                              const int32_t *parent, float *o_tree,
+                              float *lse_tree, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Debug export of the prefix split-KV partials alone.  o_part fp32
+ * [B][Hq][T][S][D] (each normalised over its chunk), lse_part fp32
+ * [B][Hq][T][S] (natural log; -inf for an empty chunk).  Chunk c covers
+ * prefix keys [c*C, (c+1)*C) clipped to [0, L_b), C = chunk size the
+ * library derives from L_cap and S (a multiple of 128).  num_splits 0 =
+ * default.  Writes S to *num_splits_out if non-NULL.
+ */
+LONGSPEC_HTA_API int longspec_hta_prefix_partial(const longspec_hta_dims *dims, const void *q,
+                                const void *k_prefix, const void *v_prefix,
+                                const int32_t *prefix_len, float *o_part,
+                                float *lse_part, int num_splits,
+                                int prefix_kernel, int *num_splits_out,
+                                void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
+/* Synchronises `stream`, reads and clears the status word of `workspace`,
+ * and returns LONGSPEC_HTA_OK or the first device-detected error. */
+LONGSPEC_HTA_API int longspec_hta_get_status(void *workspace, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LONGSPEC_HTA_H */

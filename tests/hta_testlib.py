@@ -1,0 +1,82 @@
+"""Shared helpers of the GPU parity tests: input placement, oracle calls and
+the parity gates.
+
+Gates (fp32 accumulation over bf16 inputs, out rounded to bf16):
+  * out: max |gpu - oracle| <= 1e-2 and mean |gpu - oracle| <= 1e-3;
+  * lse: max |gpu - oracle| <= 1e-3 (natural log);
+  * out, per row: ||gpu - oracle||_2 / ||oracle||_2 <= 2e-2.  The two
+    absolute gates alone are blind at 32k keys, where |out| ~ 1e-2 and the
+    tree's share of the softmax mass is ~1e-4; the per-row relative gate and
+    the separate tree-partial comparison are not.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from tree_masked_verification_b200.inputs import Workload, bf16_bits
+
+OUT_MAX_ABS = 1e-2
+OUT_MEAN_ABS = 1e-3
+LSE_ABS = 1e-3
+ROW_REL_L2 = 2e-2
+
+
+def to_device(inp: dict, device="cuda") -> dict:
+    return {k: v.to(device).contiguous() for k, v in inp.items()}
+
+
+def oracle_problem(inp: dict, scale: float = 0.0) -> oracle.Problem:
+    return oracle.Problem(
+        bf16_bits(inp["q"]), bf16_bits(inp["k_prefix"]), bf16_bits(inp["v_prefix"]),
+        inp["prefix_len"].cpu().numpy(), bf16_bits(inp["k_tree"]),
+        bf16_bits(inp["v_tree"]), inp["parent"].cpu().numpy(), scale=scale)
+
+
+def assert_parity(out, lse, out_ref, lse_ref, what=""):
+    """out/lse: GPU results (any shape, row-major rows of D); *_ref: fp64."""
+    o = np.asarray(out.detach().float().cpu().numpy(), dtype=np.float64)
+    l = np.asarray(lse.detach().float().cpu().numpy(), dtype=np.float64)
+    o_ref = np.asarray(out_ref, dtype=np.float64).reshape(o.shape)
+    l_ref = np.asarray(lse_ref, dtype=np.float64).reshape(l.shape)
+    assert np.isfinite(o).all() and np.isfinite(l).all(), f"{what}: non-finite output"
+    d = np.abs(o - o_ref)
+    D = o.shape[-1]
+    rows_err = np.linalg.norm((o - o_ref).reshape(-1, D), axis=1)
+    rows_ref = np.maximum(np.linalg.norm(o_ref.reshape(-1, D), axis=1), 1e-6)
+    rel = (rows_err / rows_ref).max()
+    lse_err = np.abs(l - l_ref).max()
+    msg = (f"{what}: out max {d.max():.3e} mean {d.mean():.3e} row-rel {rel:.3e} "
+           f"lse {lse_err:.3e}")
+    assert d.max() <= OUT_MAX_ABS, msg
+    assert d.mean() <= OUT_MEAN_ABS, msg
+    assert lse_err <= LSE_ABS, msg
+    assert rel <= ROW_REL_L2, msg
+    return dict(max_abs=float(d.max()), mean_abs=float(d.mean()), row_rel=float(rel),
+                lse_abs=float(lse_err))
+
+
+def sample_rows(w: Workload, n_heads: int = 3):
+    """(b, kvh, [(g, t), ...]) samples covering tile edges of the packed rows
+    r = g*T + t (0, 1, 63/64, 127/128, 255/256, the last row)."""
+    M = w.G * w.T
+    picks = sorted({r for r in (0, 1, 63, 64, 127, 128, 200, 255, 256, 300, M - 2, M - 1)
+                    if 0 <= r < M})
+    heads = [(0, 0), (w.B - 1, w.Hkv - 1), (w.B // 2, w.Hkv // 2)][:n_heads]
+    out = []
+    for b, kvh in dict.fromkeys(heads):
+        out.append((b, kvh, [(r // w.T, r % w.T) for r in picks]))
+    return out
+
+
+def oracle_rows_for_head(w: Workload, b: int, kvh: int, gts):
+    """Oracle out/lse of rows (b, kvh*G + g, t) using only that head's inputs."""
+    inp = w.generate_head(b, kvh)
+    p = oracle_problem(inp, w.scale)
+    rows = np.array([[0, g, t] for g, t in gts], dtype=np.int32)
+    return p.attention(rows)
+
+
+def make_inputs(w: Workload, device="cuda") -> dict:
+    return to_device(w.generate(), device)

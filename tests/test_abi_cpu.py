@@ -1,0 +1,113 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol
+the header declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from tree_masked_verification_b200 import build, hta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "longspec_hta.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return hta.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LONGSPEC_HTA_API\s+[\w\s\*]+?\b(longspec_hta_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    assert "longspec_hta_verify" in names and len(names) >= 10
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", hta.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\b(longspec_hta_\w+)\b", out))
+    missing = [n for n in declared_symbols() if n not in exported]
+    assert not missing, missing
+    assert sorted(exported) == sorted(set(hta.EXPORTED)), "binding list out of date"
+
+
+def test_header_is_plain_c():
+    subprocess.run(["gcc", "-fsyntax-only", "-std=c99", "-x", "c", "-I/usr/local/cuda/include",
+                    HEADER], check=True)
+
+
+def test_abi_version_and_strerror(lib):
+    assert lib.longspec_hta_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -16, -17, -18, 12345):
+        assert lib.longspec_hta_strerror(code)
+
+
+def _dims(**kw):
+    d = dict(B=1, Hq=32, Hkv=8, D=128, T=68, L_cap=32768, scale=0.0)
+    d.update(kw)
+    return hta.Dims(d["B"], d["Hq"], d["Hkv"], d["D"], d["T"], d["L_cap"], d["scale"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=30), hta.ERR_INVALID_DIMS),
+    (dict(D=96), hta.ERR_UNSUPPORTED_D),
+    (dict(T=257), hta.ERR_T_TOO_LARGE),
+    (dict(T=0), hta.ERR_INVALID_DIMS),
+    (dict(scale=-1.0), hta.ERR_INVALID_DIMS),
+    (dict(L_cap=-1), hta.ERR_INVALID_DIMS),
+    (dict(B=1 << 20, Hkv=8, Hq=8), hta.ERR_INVALID_DIMS),
+])
+def test_verify_rejects_bad_dims_on_host(lib, kw, code):
+    d = _dims(**kw)
+    rc = lib.longspec_hta_verify(ctypes.byref(d), *([16] * 9), 16, 1 << 30, None)
+    assert rc == code
+
+
+def test_verify_rejects_null_and_misaligned_on_host(lib):
+    d = _dims()
+    ptrs = [4096 * (i + 1) for i in range(9)]
+    for i in range(9):
+        bad = list(ptrs)
+        bad[i] = 0
+        assert lib.longspec_hta_verify(ctypes.byref(d), *bad, 4096 * 20, 1 << 30, None) == hta.ERR_NULL_POINTER
+        bad[i] = ptrs[i] + 8
+        assert lib.longspec_hta_verify(ctypes.byref(d), *bad, 4096 * 20, 1 << 30, None) == hta.ERR_MISALIGNED
+
+
+def test_verify_ex_rejects_bad_options(lib):
+    d = _dims()
+    for opts in (hta.Options(-1, 0, None, None), hta.Options(0, 7, None, None)):
+        rc = lib.longspec_hta_verify_ex(ctypes.byref(d), *[4096 * (i + 1) for i in range(9)],
+                                        4096 * 20, 1 << 30, ctypes.byref(opts), None)
+        assert rc == hta.ERR_INVALID_OPTION
+
+
+@pytest.mark.parametrize("L_cap,req,S,chunk", [
+    (32768, 6, 6, 43 * 128),
+    (32768, 1, 1, 32768),
+    (256, 6, 2, 128),
+    (1000, 3, 3, 384),
+    (0, 4, 1, 128),
+    (262144, 64, 64, 4096),
+])
+def test_chunking_arithmetic(lib, L_cap, req, S, chunk):
+    got = hta.chunking(_dims(L_cap=L_cap), req)
+    assert got == (S, chunk)
+    # chunks cover [0, L_cap) exactly once
+    assert (S - 1) * chunk < max(L_cap, 1) <= S * chunk
+
+
+def test_workspace_bytes_formula(lib):
+    d = _dims()
+    n = hta.workspace_bytes(d, 6)
+    rows = 1 * 32 * 68
+    assert n >= 256 + rows * 6 * 129 * 4
+    assert n - (256 + rows * 6 * 129 * 4) < 1024

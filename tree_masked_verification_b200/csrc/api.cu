@@ -1,0 +1,505 @@
+// api.cu -- the C ABI of liblongspec_hta.so (declared in include/longspec_hta.h).
+//
+// Host side only: argument checks, the split-KV chunking, tensor-map
+// (TMA descriptor) encoding with a small per-pointer cache, and the two
+// launches of one verification call (prefix kernel, then the tree pass fused
+// with the log-sum-exp merge).  Nothing here computes attention.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/longspec_hta.h"
+#include "hta_kernels.h"
+
+using hta::PrefixParams;
+using hta::TreeMergeParams;
+
+namespace {
+
+// ---------------------------------------------------------------- device
+struct DeviceInfo {
+    bool probed = false;
+    bool supported = false;
+    int num_sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(DeviceInfo *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return LONGSPEC_HTA_ERR_CUDA;
+        d.supported = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        d.probed = true;
+    }
+    *out = d;
+    return d.supported ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE;
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct MapKey {
+    int dev;
+    const void *ptr;
+    uint64_t rows;
+    int D;
+    bool operator==(const MapKey &o) const {
+        return dev == o.dev && ptr == o.ptr && rows == o.rows && D == o.D;
+    }
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+constexpr int kMapCache = 48;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mu;
+
+// [rows][D] bf16 matrix as 64-column x 128-row boxes with 128-byte swizzle.
+int tensor_map(const void *ptr, uint64_t rows, int D, CUtensorMap *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    const MapKey key{dev, ptr, rows, D};
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (auto &e : g_maps)
+        if (e.used && e.key == key) { *out = e.map; return LONGSPEC_HTA_OK; }
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return LONGSPEC_HTA_ERR_CUDA;
+    CUtensorMap m;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return LONGSPEC_HTA_ERR_CUDA;
+    MapEntry &e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.key = key;
+    e.map = m;
+    e.used = true;
+    *out = m;
+    return LONGSPEC_HTA_OK;
+}
+
+// ------------------------------------------------------------- validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const longspec_hta_dims *d) {
+    if (!d) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->T < 1 || d->L_cap < 0 || d->Hq % d->Hkv != 0)
+        return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    if (!(d->scale >= 0.f) || std::isinf(d->scale)) return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    if (d->D != 64 && d->D != 128) return LONGSPEC_HTA_ERR_UNSUPPORTED_D;
+    if (d->T > LONGSPEC_HTA_T_MAX) return LONGSPEC_HTA_ERR_T_TOO_LARGE;
+    const long long rows = 1LL * d->B * d->Hq * d->T;
+    const long long keys = 1LL * d->B * d->Hkv * d->L_cap;
+    if (rows >= (1LL << 31) || keys + 128 >= (1LL << 31) || 1LL * d->B * d->Hkv > 65535)
+        return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    return LONGSPEC_HTA_OK;
+}
+
+float scale_of(const longspec_hta_dims *d) {
+    return d->scale > 0.f ? d->scale : 1.f / std::sqrt(static_cast<float>(d->D));
+}
+
+int m_tiles_of(const longspec_hta_dims *d) {
+    const int M = (d->Hq / d->Hkv) * d->T;
+    return (M + 127) / 128;
+}
+
+// Split-KV chunking: chunk_tiles tiles of 128 keys per split, S splits.
+struct Chunking {
+    int S, chunk_tiles;
+};
+
+Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms) {
+    const int tiles = std::max(1, (d->L_cap + hta::kKeyTile - 1) / hta::kKeyTile);
+    auto make = [&](int s) {
+        s = std::max(1, std::min(s, tiles));
+        const int ct = (tiles + s - 1) / s;
+        return Chunking{(tiles + ct - 1) / ct, ct};
+    };
+    if (requested > 0) return make(requested);
+    // smallest estimated time: waves of CTAs x (tiles per CTA + fixed cost)
+    const long long units = 1LL * d->B * d->Hkv * m_tiles_of(d);
+    Chunking best = make(1);
+    double best_cost = 1e300;
+    for (int s = 1; s <= std::min(tiles, 64); ++s) {
+        const Chunking c = make(s);
+        const long long ctas = units * c.S;
+        const long long waves = (ctas + num_sms - 1) / std::max(1, num_sms);
+        const double cost = waves * (c.chunk_tiles + 2.0) + 0.05 * c.S;
+        if (cost < best_cost - 1e-9) { best_cost = cost; best = c; }
+    }
+    return best;
+}
+
+struct WsLayout {
+    size_t o_off, lse_off, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const longspec_hta_dims *d, int S) {
+    const size_t rows = 1ull * d->B * d->Hq * d->T;
+    WsLayout w;
+    w.o_off = hta::kStatusBytes;
+    w.lse_off = align256(w.o_off + rows * S * d->D * sizeof(float));
+    w.total = align256(w.lse_off + rows * S * sizeof(float));
+    return w;
+}
+
+PrefixParams prefix_params(const longspec_hta_dims *d, const Chunking &c, const void *q,
+                           const void *kp, const void *vp, const int32_t *plen, float *o_part,
+                           float *lse_part, uint32_t *status) {
+    PrefixParams p{};
+    p.B = d->B; p.Hq = d->Hq; p.Hkv = d->Hkv; p.D = d->D; p.T = d->T; p.L_cap = d->L_cap;
+    p.G = d->Hq / d->Hkv;
+    p.M = p.G * d->T;
+    p.m_tiles = (p.M + 127) / 128;
+    p.S = c.S;
+    p.chunk_tiles = c.chunk_tiles;
+    p.scale_log2 = scale_of(d) * hta::kLog2e;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k_prefix = static_cast<const __nv_bfloat16 *>(kp);
+    p.v_prefix = static_cast<const __nv_bfloat16 *>(vp);
+    p.prefix_len = plen;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.status = status;
+    return p;
+}
+
+int run_prefix(const longspec_hta_dims *d, const PrefixParams &p, int kernel, cudaEvent_t ev_begin,
+               cudaEvent_t ev_end, cudaStream_t stream) {
+    CUtensorMap tq, tk, tv;
+    if (kernel == LONGSPEC_HTA_PREFIX_TCGEN05) {
+        const uint64_t qrows = 1ull * d->B * d->Hq * d->T;
+        const uint64_t krows = 1ull * d->B * d->Hkv * std::max(d->L_cap, 1);
+        int rc;
+        if ((rc = tensor_map(p.q, qrows, d->D, &tq)) != LONGSPEC_HTA_OK) return rc;
+        if ((rc = tensor_map(p.k_prefix, krows, d->D, &tk)) != LONGSPEC_HTA_OK) return rc;
+        if ((rc = tensor_map(p.v_prefix, krows, d->D, &tv)) != LONGSPEC_HTA_OK) return rc;
+    }
+    if (ev_begin && cudaEventRecord(ev_begin, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    cudaError_t e = (kernel == LONGSPEC_HTA_PREFIX_TCGEN05)
+                        ? hta::launch_prefix_tc(p, tq, tk, tv, stream)
+                        : hta::launch_prefix_simt(p, stream);
+    if (e != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    if (ev_end && cudaEventRecord(ev_end, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    return LONGSPEC_HTA_OK;
+}
+
+TreeMergeParams tree_params(const longspec_hta_dims *d, int mode, int S, const void *q,
+                            const void *kt, const void *vt, const int32_t *parent,
+                            const int32_t *plen, const float *o_part, const float *lse_part,
+                            uint32_t *status) {
+    TreeMergeParams t{};
+    t.B = d->B; t.Hq = d->Hq; t.Hkv = d->Hkv; t.D = d->D; t.T = d->T; t.L_cap = d->L_cap;
+    t.S = S;
+    t.scale_log2 = scale_of(d) * hta::kLog2e;
+    t.mode = mode;
+    t.q = static_cast<const __nv_bfloat16 *>(q);
+    t.k_tree = static_cast<const __nv_bfloat16 *>(kt);
+    t.v_tree = static_cast<const __nv_bfloat16 *>(vt);
+    t.parent = parent;
+    t.prefix_len = plen;
+    t.o_part = o_part;
+    t.lse_part = lse_part;
+    t.status = status;
+    return t;
+}
+
+}  // namespace
+
+extern "C" {
+
+int longspec_hta_abi_version(void) { return LONGSPEC_HTA_ABI_VERSION; }
+
+const char *longspec_hta_strerror(int code) {
+    switch (code) {
+    case LONGSPEC_HTA_OK: return "ok";
+    case LONGSPEC_HTA_ERR_INVALID_DIMS: return "invalid dimensions or scale";
+    case LONGSPEC_HTA_ERR_NULL_POINTER: return "null pointer";
+    case LONGSPEC_HTA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case LONGSPEC_HTA_ERR_T_TOO_LARGE: return "tree larger than LONGSPEC_HTA_T_MAX";
+    case LONGSPEC_HTA_ERR_UNSUPPORTED_D: return "head dimension must be 64 or 128";
+    case LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case LONGSPEC_HTA_ERR_CUDA: return "CUDA call failed";
+    case LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+    case LONGSPEC_HTA_ERR_INVALID_OPTION: return "invalid option";
+    case LONGSPEC_HTA_ERR_BAD_PARENT: return "parent[i] outside [-1, i)";
+    case LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE: return "prefix_len outside [0, L_cap]";
+    case LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT: return "in-kernel wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int longspec_hta_default_splits(const longspec_hta_dims *dims) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    DeviceInfo di;
+    rc = current_device(&di);
+    if (rc) return rc;
+    return chunking_for(dims, 0, di.num_sms).S;
+}
+
+int longspec_hta_chunking(const longspec_hta_dims *dims, int num_splits, int *num_splits_out,
+                          int *chunk_keys_out) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (num_splits < 0) return LONGSPEC_HTA_ERR_INVALID_OPTION;
+    int sms = 148;
+    if (num_splits == 0) {
+        DeviceInfo di;
+        if ((rc = current_device(&di))) return rc;
+        sms = di.num_sms;
+    }
+    const Chunking c = chunking_for(dims, num_splits, sms);
+    if (num_splits_out) *num_splits_out = c.S;
+    if (chunk_keys_out) *chunk_keys_out = c.chunk_tiles * hta::kKeyTile;
+    return LONGSPEC_HTA_OK;
+}
+
+size_t longspec_hta_workspace_bytes(const longspec_hta_dims *dims, int num_splits) {
+    if (check_dims(dims) != LONGSPEC_HTA_OK || num_splits < 0) return 0;
+    int sms = 148;
+    if (num_splits == 0) {
+        DeviceInfo di;
+        if (current_device(&di) != LONGSPEC_HTA_OK) return 0;
+        sms = di.num_sms;
+    }
+    return ws_layout(dims, chunking_for(dims, num_splits, sms).S).total;
+}
+
+int longspec_hta_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    if (!aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    return cudaMemsetAsync(workspace, 0, hta::kStatusBytes, stream) == cudaSuccess ? LONGSPEC_HTA_OK
+                                                                                  : LONGSPEC_HTA_ERR_CUDA;
+}
+
+int longspec_hta_verify_ex(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                           const void *v_prefix, const int32_t *prefix_len, const void *k_tree,
+                           const void *v_tree, const int32_t *parent, void *out, float *lse,
+                           void *workspace, size_t workspace_bytes,
+                           const longspec_hta_options *opts, cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, out, lse, workspace};
+    for (const void *p : ptrs) {
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    longspec_hta_options o{};
+    if (opts) o = *opts;
+    if (o.num_splits < 0 || (o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
+                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
+        return LONGSPEC_HTA_ERR_INVALID_OPTION;
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms);
+    const WsLayout w = ws_layout(dims, c.S);
+    if (workspace_bytes < w.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    float *o_part = reinterpret_cast<float *>(ws + w.o_off);
+    float *lse_part = reinterpret_cast<float *>(ws + w.lse_off);
+
+    const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part, status);
+    if ((rc = run_prefix(dims, pp, o.prefix_kernel, o.prefix_begin, o.prefix_end, stream))) return rc;
+    TreeMergeParams tp = tree_params(dims, hta::kTreeModeMerge, c.S, q, k_tree, v_tree, parent,
+                                     prefix_len, o_part, lse_part, status);
+    tp.out = static_cast<__nv_bfloat16 *>(out);
+    tp.lse = lse;
+    return hta::launch_tree_merge(tp, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
+int longspec_hta_verify(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                        const void *v_prefix, const int32_t *prefix_len, const void *k_tree,
+                        const void *v_tree, const int32_t *parent, void *out, float *lse,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return longspec_hta_verify_ex(dims, q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent,
+                                  out, lse, workspace, workspace_bytes, nullptr, stream);
+}
+
+// ---- end-to-end call on host buffers -------------------------------------
+namespace {
+struct ArenaLayout {
+    size_t q, kp, vp, plen, kt, vt, par, out, lse, ws, total;
+    size_t q_b, kv_b, plen_b, tree_b, par_b, out_b, lse_b, ws_b;
+};
+
+ArenaLayout arena_layout(const longspec_hta_dims *d, int num_sms) {
+    ArenaLayout a{};
+    a.q_b = 2ull * d->B * d->Hq * d->T * d->D;
+    a.kv_b = 2ull * d->B * d->Hkv * d->L_cap * d->D;
+    a.plen_b = 4ull * d->B;
+    a.tree_b = 2ull * d->B * d->Hkv * d->T * d->D;
+    a.par_b = 4ull * d->B * d->T;
+    a.out_b = a.q_b;
+    a.lse_b = 4ull * d->B * d->Hq * d->T;
+    a.ws_b = ws_layout(d, chunking_for(d, 0, num_sms).S).total;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align256(off + std::max<size_t>(bytes, 1)); return o; };
+    a.q = take(a.q_b); a.kp = take(a.kv_b); a.vp = take(a.kv_b); a.plen = take(a.plen_b);
+    a.kt = take(a.tree_b); a.vt = take(a.tree_b); a.par = take(a.par_b);
+    a.out = take(a.out_b); a.lse = take(a.lse_b); a.ws = take(a.ws_b);
+    a.total = off;
+    return a;
+}
+}  // namespace
+
+size_t longspec_hta_host_arena_bytes(const longspec_hta_dims *dims) {
+    if (check_dims(dims) != LONGSPEC_HTA_OK) return 0;
+    DeviceInfo di;
+    if (current_device(&di) != LONGSPEC_HTA_OK) return 0;
+    return arena_layout(dims, di.num_sms).total;
+}
+
+int longspec_hta_verify_host(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                             const void *v_prefix, const int32_t *prefix_len, const void *k_tree,
+                             const void *v_tree, const int32_t *parent, void *out, float *lse,
+                             void *arena, size_t arena_bytes, cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, out, lse, arena};
+    for (const void *p : ptrs)
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    if (!aligned16(arena)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    const ArenaLayout a = arena_layout(dims, di.num_sms);
+    if (arena_bytes < a.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *base = static_cast<uint8_t *>(arena);
+    struct Copy { size_t off; const void *src; size_t bytes; };
+    const Copy ins[] = {{a.q, q, a.q_b}, {a.kp, k_prefix, a.kv_b}, {a.vp, v_prefix, a.kv_b},
+                        {a.plen, prefix_len, a.plen_b}, {a.kt, k_tree, a.tree_b},
+                        {a.vt, v_tree, a.tree_b}, {a.par, parent, a.par_b}};
+    for (const Copy &c : ins)
+        if (c.bytes && cudaMemcpyAsync(base + c.off, c.src, c.bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return LONGSPEC_HTA_ERR_CUDA;
+    if (cudaMemsetAsync(base + a.ws, 0, hta::kStatusBytes, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    rc = longspec_hta_verify(dims, base + a.q, base + a.kp, base + a.vp,
+                             reinterpret_cast<const int32_t *>(base + a.plen), base + a.kt, base + a.vt,
+                             reinterpret_cast<const int32_t *>(base + a.par), base + a.out,
+                             reinterpret_cast<float *>(base + a.lse), base + a.ws, a.ws_b, stream);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(out, base + a.out, a.out_b, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaMemcpyAsync(lse, base + a.lse, a.lse_b, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return LONGSPEC_HTA_ERR_CUDA;
+    return LONGSPEC_HTA_OK;
+}
+
+// ---- debug exports --------------------------------------------------------
+int longspec_hta_tree_mask(const int32_t *parent, int B, int T, uint32_t *bits, void *workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
+    if (!parent || !bits || !workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    if (!aligned16(parent) || !aligned16(bits) || !aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    if (B < 1 || B > 65535 || T < 1) return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    if (T > LONGSPEC_HTA_T_MAX) return LONGSPEC_HTA_ERR_T_TOO_LARGE;
+    if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo di;
+    int rc = current_device(&di);
+    if (rc) return rc;
+    TreeMergeParams t{};
+    t.B = B; t.Hq = 1; t.Hkv = 1; t.D = 128; t.T = T;
+    t.mode = hta::kTreeModeMask;
+    t.parent = parent;
+    t.mask_out = bits;
+    t.status = static_cast<uint32_t *>(workspace);
+    return hta::launch_tree_merge(t, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
+int longspec_hta_tree_partial(const longspec_hta_dims *dims, const void *q, const void *k_tree,
+                              const void *v_tree, const int32_t *parent, float *o_tree,
+                              float *lse_tree, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const void *ptrs[] = {q, k_tree, v_tree, parent, o_tree, lse_tree, workspace};
+    for (const void *p : ptrs) {
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    TreeMergeParams t = tree_params(dims, hta::kTreeModePartial, 0, q, k_tree, v_tree, parent, nullptr,
+                                    nullptr, nullptr, static_cast<uint32_t *>(workspace));
+    t.o_tree = o_tree;
+    t.lse_tree = lse_tree;
+    return hta::launch_tree_merge(t, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
+int longspec_hta_prefix_partial(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                                const void *v_prefix, const int32_t *prefix_len, float *o_part,
+                                float *lse_part, int num_splits, int prefix_kernel,
+                                int *num_splits_out, void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, o_part, lse_part, workspace};
+    for (const void *p : ptrs) {
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    if (num_splits < 0 || (prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
+                           prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
+        return LONGSPEC_HTA_ERR_INVALID_OPTION;
+    if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    const Chunking c = chunking_for(dims, num_splits, di.num_sms);
+    if (num_splits_out) *num_splits_out = c.S;
+    const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part,
+                                          static_cast<uint32_t *>(workspace));
+    return run_prefix(dims, pp, prefix_kernel, nullptr, nullptr, stream);
+}
+
+int longspec_hta_get_status(void *workspace, cudaStream_t stream) {
+    if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess)
+        return LONGSPEC_HTA_ERR_CUDA;
+    if (word & hta::kStatusBadParent) return LONGSPEC_HTA_ERR_BAD_PARENT;
+    if (word & hta::kStatusPrefixLenRange) return LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE;
+    if (word & hta::kStatusPipelineTimeout) return LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT;
+    return LONGSPEC_HTA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// hta_kernels.h -- parameter blocks and launchers of the Hybrid Tree
+// Attention kernels (internal to liblongspec_hta.so).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "hta_common.cuh"
+
+namespace hta {
+
+constexpr int kTreeRowsPerCta = 16;
+constexpr int kKeyTile = 128;   // keys per prefix tile; chunk sizes are multiples of it
+
+enum TreeMode : int { kTreeModeMerge = 0, kTreeModePartial = 1, kTreeModeMask = 2 };
+
+struct TreeMergeParams {
+    int B, Hq, Hkv, D, T, L_cap, S;
+    float scale_log2;                 // softmax scale * log2(e)
+    int mode;                         // TreeMode
+    const __nv_bfloat16 *q, *k_tree, *v_tree;
+    const int32_t *parent, *prefix_len;
+    const float *o_part, *lse_part;   // [rows][S][D], [rows][S] (natural log)
+    __nv_bfloat16 *out;
+    float *lse;
+    float *o_tree, *lse_tree;         // kTreeModePartial outputs
+    uint32_t *mask_out;               // kTreeModeMask output [B][T][ceil(T/32)]
+    uint32_t *status;
+};
+
+// Prefix split-KV partials.  Rows of one (b, KV head) are the packed query
+// group r = g*T + t (g < G), contiguous in q; global row index
+// (b*Hkv + kvh)*M + r equals (b*Hq + h)*T + t.
+struct PrefixParams {
+    int B, Hq, Hkv, D, T, L_cap;
+    int G, M, m_tiles;                // M = G*T, m_tiles = ceil(M / 128)
+    int S, chunk_tiles;               // split c covers keys [c, c+1) * chunk_tiles * 128
+    float scale_log2;
+    const __nv_bfloat16 *q, *k_prefix, *v_prefix;   // (SIMT kernel reads these directly)
+    const int32_t *prefix_len;
+    float *o_part, *lse_part;         // [rows][S][D], [rows][S]
+    uint32_t *status;
+};
+
+cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream);
+cudaError_t launch_prefix_simt(const PrefixParams &p, cudaStream_t stream);
+// Tensor maps: q as [B*Hq*T][D], k/v as [B*Hkv*L_cap][D], box 64 x 128, 128B swizzle.
+cudaError_t launch_prefix_tc(const PrefixParams &p, const CUtensorMap &tm_q,
+                             const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                             cudaStream_t stream);
+
+}  // namespace hta

@@ -1,0 +1,270 @@
+"""ctypes binding of liblongspec_hta.so (Hybrid Tree Attention on B200).
+
+Argument marshalling only: every step of the verification attention runs in
+the library's CUDA kernels.  Tensors are torch tensors on the current CUDA
+device; the library launches on torch's current stream unless a stream is
+given.  The library must have been built (``tree_masked_verification_b200.build``):
+there is no fallback of any kind, and a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblongspec_hta.so")
+_lock = threading.Lock()
+_lib = None
+
+OK = 0
+ERR_INVALID_DIMS = -1
+ERR_NULL_POINTER = -2
+ERR_MISALIGNED = -3
+ERR_T_TOO_LARGE = -4
+ERR_UNSUPPORTED_D = -5
+ERR_WORKSPACE_TOO_SMALL = -6
+ERR_CUDA = -7
+ERR_UNSUPPORTED_DEVICE = -8
+ERR_INVALID_OPTION = -9
+ERR_BAD_PARENT = -16
+ERR_PREFIX_LEN_RANGE = -17
+ERR_PIPELINE_TIMEOUT = -18
+
+PREFIX_TCGEN05 = 0
+PREFIX_SIMT = 1
+T_MAX = 256
+
+EXPORTED = [
+    "longspec_hta_abi_version", "longspec_hta_strerror", "longspec_hta_default_splits",
+    "longspec_hta_chunking",
+    "longspec_hta_workspace_bytes", "longspec_hta_workspace_init", "longspec_hta_verify",
+    "longspec_hta_verify_ex", "longspec_hta_host_arena_bytes", "longspec_hta_verify_host",
+    "longspec_hta_tree_mask", "longspec_hta_tree_partial", "longspec_hta_prefix_partial",
+    "longspec_hta_get_status",
+]
+
+
+class HtaError(RuntimeError):
+    def __init__(self, code: int):
+        msg = load().longspec_hta_strerror(code).decode()
+        super().__init__(f"longspec_hta error {code}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("T", ctypes.c_int), ("L_cap", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("num_splits", ctypes.c_int), ("prefix_kernel", ctypes.c_int),
+                ("prefix_begin", ctypes.c_void_p), ("prefix_end", ctypes.c_void_p)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load the library (once).  Raises if it was not built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m tree_masked_verification_b200.build` (no fallback exists)")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            pd = ctypes.POINTER(Dims)
+            lib.longspec_hta_abi_version.restype = ci
+            lib.longspec_hta_strerror.argtypes = [ci]
+            lib.longspec_hta_strerror.restype = ctypes.c_char_p
+            lib.longspec_hta_default_splits.argtypes = [pd]
+            lib.longspec_hta_workspace_bytes.argtypes = [pd, ci]
+            lib.longspec_hta_workspace_bytes.restype = sz
+            lib.longspec_hta_workspace_init.argtypes = [vp, sz, vp]
+            lib.longspec_hta_verify.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
+            lib.longspec_hta_verify_ex.argtypes = [pd] + [vp] * 9 + [vp, sz, ctypes.POINTER(Options), vp]
+            lib.longspec_hta_host_arena_bytes.argtypes = [pd]
+            lib.longspec_hta_host_arena_bytes.restype = sz
+            lib.longspec_hta_verify_host.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
+            lib.longspec_hta_tree_mask.argtypes = [vp, ci, ci, vp, vp, sz, vp]
+            lib.longspec_hta_tree_partial.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.longspec_hta_prefix_partial.argtypes = [pd, vp, vp, vp, vp, vp, vp, ci, ci,
+                                                        ctypes.POINTER(ci), vp, sz, vp]
+            lib.longspec_hta_get_status.argtypes = [vp, vp]
+            lib.longspec_hta_chunking.argtypes = [pd, ci, ctypes.POINTER(ci), ctypes.POINTER(ci)]
+            _lib = lib
+    return _lib
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise HtaError(rc)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def dims_of(q: torch.Tensor, k_prefix: torch.Tensor, scale: float = 0.0) -> Dims:
+    B, Hq, T, D = q.shape
+    return Dims(B, Hq, k_prefix.shape[1], D, T, k_prefix.shape[2], float(scale))
+
+
+def _need(t: torch.Tensor, name: str, dtype, device=None):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+
+
+def default_splits(dims: Dims) -> int:
+    rc = load().longspec_hta_default_splits(ctypes.byref(dims))
+    if rc < 0:
+        raise HtaError(rc)
+    return rc
+
+
+def chunking(dims: Dims, num_splits: int = 0):
+    """(S, chunk_keys) the library uses for a requested split count."""
+    S, C = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().longspec_hta_chunking(ctypes.byref(dims), int(num_splits), ctypes.byref(S),
+                                        ctypes.byref(C)))
+    return S.value, C.value
+
+
+def workspace_bytes(dims: Dims, num_splits: int = 0) -> int:
+    n = load().longspec_hta_workspace_bytes(ctypes.byref(dims), int(num_splits))
+    if n == 0:
+        raise HtaError(ERR_INVALID_DIMS)
+    return n
+
+
+def new_workspace(dims: Dims, num_splits: int = 0, device=None) -> torch.Tensor:
+    """A zeroed device workspace for verify (status word cleared)."""
+    return torch.zeros(workspace_bytes(dims, num_splits), dtype=torch.uint8,
+                       device=device or torch.device("cuda"))
+
+
+def verify(q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, *, out=None,
+           lse=None, workspace=None, scale: float = 0.0, num_splits: int = 0,
+           prefix_kernel: int = PREFIX_TCGEN05, prefix_events=None, stream=None):
+    """Hybrid Tree Attention of one layer.  Returns (out bf16, lse fp32)."""
+    dev = q.device
+    for t, n in ((q, "q"), (k_prefix, "k_prefix"), (v_prefix, "v_prefix"),
+                 (k_tree, "k_tree"), (v_tree, "v_tree")):
+        _need(t, n, torch.bfloat16, dev)
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    _need(parent, "parent", torch.int32, dev)
+    dims = dims_of(q, k_prefix, scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(dims, num_splits, dev)
+    opts = Options(int(num_splits), int(prefix_kernel),
+                   prefix_events[0].cuda_event if prefix_events else None,
+                   prefix_events[1].cuda_event if prefix_events else None)
+    rc = load().longspec_hta_verify_ex(
+        ctypes.byref(dims), _ptr(q), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_len),
+        _ptr(k_tree), _ptr(v_tree), _ptr(parent), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.byref(opts), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def host_arena_bytes(dims: Dims) -> int:
+    n = load().longspec_hta_host_arena_bytes(ctypes.byref(dims))
+    if n == 0:
+        raise HtaError(ERR_INVALID_DIMS)
+    return n
+
+
+def verify_host(q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, out, lse,
+                arena, *, scale: float = 0.0, stream=None):
+    """End-to-end call on host tensors (pinned for asynchronous copies): the
+    library copies inputs into the device `arena`, runs, and copies out/lse
+    back on `stream`.  Synchronise the stream before reading out/lse."""
+    for t, n in ((q, "q"), (k_prefix, "k_prefix"), (v_prefix, "v_prefix"),
+                 (k_tree, "k_tree"), (v_tree, "v_tree"), (out, "out")):
+        _need(t, n, torch.bfloat16, torch.device("cpu"))
+    _need(prefix_len, "prefix_len", torch.int32, torch.device("cpu"))
+    _need(parent, "parent", torch.int32, torch.device("cpu"))
+    _need(lse, "lse", torch.float32, torch.device("cpu"))
+    dims = dims_of(q, k_prefix, scale)
+    rc = load().longspec_hta_verify_host(
+        ctypes.byref(dims), _ptr(q), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_len),
+        _ptr(k_tree), _ptr(v_tree), _ptr(parent), _ptr(out), _ptr(lse), _ptr(arena),
+        arena.numel() * arena.element_size(), _stream(stream))
+    _check(rc)
+
+
+def tree_mask(parent: torch.Tensor, workspace=None, stream=None) -> torch.Tensor:
+    """Ancestor-or-self bits uint32-as-int32 [B][T][ceil(T/32)] (debug export)."""
+    _need(parent, "parent", torch.int32)
+    B, T = parent.shape
+    W = (T + 31) // 32
+    bits = torch.empty(B, T, W, dtype=torch.int32, device=parent.device)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=parent.device)
+    _check(load().longspec_hta_tree_mask(_ptr(parent), B, T, _ptr(bits), _ptr(workspace),
+                                         workspace.numel(), _stream(stream)))
+    return bits
+
+
+def tree_partial(q, k_tree, v_tree, parent, *, scale: float = 0.0, workspace=None, stream=None):
+    """Tree-only partial (debug export): (o_tree fp32 [B][Hq][T][D], lse_tree fp32)."""
+    B, Hq, T, D = q.shape
+    dims = Dims(B, Hq, k_tree.shape[1], D, T, 0, float(scale))
+    o = torch.empty(B, Hq, T, D, dtype=torch.float32, device=q.device)
+    l = torch.empty(B, Hq, T, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    _check(load().longspec_hta_tree_partial(ctypes.byref(dims), _ptr(q), _ptr(k_tree),
+                                            _ptr(v_tree), _ptr(parent), _ptr(o), _ptr(l),
+                                            _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, l
+
+
+def prefix_partial(q, k_prefix, v_prefix, prefix_len, *, scale: float = 0.0,
+                   num_splits: int = 0, prefix_kernel: int = PREFIX_TCGEN05,
+                   workspace=None, stream=None):
+    """Split-KV prefix partials (debug export):
+    (o_part fp32 [B][Hq][T][S][D], lse_part fp32 [B][Hq][T][S], chunk keys)."""
+    dims = dims_of(q, k_prefix, scale)
+    lib = load()
+    S, chunk_keys = chunking(dims, num_splits)
+    S_out = ctypes.c_int(0)
+    B, Hq, T, D = q.shape
+    o = torch.empty(B, Hq, T, S, D, dtype=torch.float32, device=q.device)
+    l = torch.empty(B, Hq, T, S, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    _check(lib.longspec_hta_prefix_partial(ctypes.byref(dims), _ptr(q), _ptr(k_prefix),
+                                           _ptr(v_prefix), _ptr(prefix_len), _ptr(o), _ptr(l),
+                                           int(num_splits), int(prefix_kernel), ctypes.byref(S_out),
+                                           _ptr(workspace), workspace.numel(), _stream(stream)))
+    if S_out.value != S:
+        raise RuntimeError(f"split count mismatch: library {S_out.value}, binding {S}")
+    return o, l, chunk_keys
+
+
+def get_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise, read and clear the device status word; returns the code."""
+    return int(load().longspec_hta_get_status(_ptr(workspace), _stream(stream)))
