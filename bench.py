@@ -255,6 +255,9 @@ def run_ours(args, world, rank, local):
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    for a, b in ev:          # torch creates the CUDA event on first record
+        a.record(stream)
+        b.record(stream)
     sampler = ClockSampler(local if world > 1 else 0)
     sampler.start()
     time.sleep(0.3)

@@ -2,7 +2,11 @@
 the parity gates.
 
 Gates (fp32 accumulation over bf16 inputs, out rounded to bf16):
-  * out: max |gpu - oracle| <= 1e-2 and mean |gpu - oracle| <= 1e-3;
+  * out: max |gpu - oracle| <= 1e-2 + h(oracle) and mean |gpu - oracle|
+    <= 1e-3, where h(x) is half the bf16 spacing at x: the result is
+    returned in bf16, and rounding the exact value alone moves it by up to
+    h(x) (0.0078 for |x| in [2, 4)), so the 1e-2 bound is applied to the
+    value before that final rounding;
   * lse: max |gpu - oracle| <= 1e-3 (natural log);
   * out, per row: ||gpu - oracle||_2 / ||oracle||_2 <= 2e-2.  The two
     absolute gates alone are blind at 32k keys, where |out| ~ 1e-2 and the
@@ -34,6 +38,13 @@ def oracle_problem(inp: dict, scale: float = 0.0) -> oracle.Problem:
         bf16_bits(inp["v_tree"]), inp["parent"].cpu().numpy(), scale=scale)
 
 
+def bf16_half_ulp(x) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |x| (bf16 keeps 8 of float32's 24
+    significand bits, so its spacing is float32's times 2^16)."""
+    x32 = np.abs(np.asarray(x, dtype=np.float32))
+    return np.spacing(x32).astype(np.float64) * 2.0 ** 15
+
+
 def assert_parity(out, lse, out_ref, lse_ref, what=""):
     """out/lse: GPU results (any shape, row-major rows of D); *_ref: fp64."""
     o = np.asarray(out.detach().float().cpu().numpy(), dtype=np.float64)
@@ -42,14 +53,16 @@ def assert_parity(out, lse, out_ref, lse_ref, what=""):
     l_ref = np.asarray(lse_ref, dtype=np.float64).reshape(l.shape)
     assert np.isfinite(o).all() and np.isfinite(l).all(), f"{what}: non-finite output"
     d = np.abs(o - o_ref)
+    half_ulp = bf16_half_ulp(o_ref) if out.dtype == torch.bfloat16 else np.zeros_like(o_ref)
+    excess = d - (OUT_MAX_ABS + half_ulp)
     D = o.shape[-1]
     rows_err = np.linalg.norm((o - o_ref).reshape(-1, D), axis=1)
     rows_ref = np.maximum(np.linalg.norm(o_ref.reshape(-1, D), axis=1), 1e-6)
     rel = (rows_err / rows_ref).max()
     lse_err = np.abs(l - l_ref).max()
-    msg = (f"{what}: out max {d.max():.3e} mean {d.mean():.3e} row-rel {rel:.3e} "
-           f"lse {lse_err:.3e}")
-    assert d.max() <= OUT_MAX_ABS, msg
+    msg = (f"{what}: out max {d.max():.3e} (over bound {excess.max():.3e}) mean {d.mean():.3e} "
+           f"row-rel {rel:.3e} lse {lse_err:.3e}")
+    assert excess.max() <= 0, msg
     assert d.mean() <= OUT_MEAN_ABS, msg
     assert lse_err <= LSE_ABS, msg
     assert rel <= ROW_REL_L2, msg
