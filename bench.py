@@ -59,6 +59,24 @@ def workload_config(w, S, n_sets):
             if n_sets > 1 else "K/V bytes per call > 2x L2"}
 
 
+def profiled_traffic(workload_name, kernel_file="tree_masked_verification_b200/csrc/prefix_tc.cu"):
+    """DRAM bytes per launch of the prefix kernel from the committed ncu
+    summary, if that summary was taken on this workload with the current
+    kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"prefix_tc_kernel_{workload_name}.json")
+    try:
+        with open(path) as f:
+            prof = json.load(f)
+        with open(os.path.join(ROOT, kernel_file), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except (OSError, ValueError):
+        return None
+    if prof.get("source_sha256_16") != sha:
+        return None
+    return int(prof["dram_bytes_read"] + prof["dram_bytes_write"])
+
+
 def prefix_algorithmic_bytes(w):
     """Bytes the prefix kernel must move at minimum: K and V of the L_b
     prefix keys of every (b, KV head) (2 * D * 2 bytes per key and head),
@@ -298,7 +316,7 @@ def run_ours(args, world, rank, local):
         "config": workload_config(w, S, n_sets),
         "roofline": {"bound": "hbm", "kernel": "prefix_tc_kernel", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": profiled_traffic(w.name),
                      "algorithmic_bytes": pbytes, "avg_launch_us": prefix_avg_ms * 1e3},
         "call_roofline": {"bytes": call_bytes, "achieved_gbs": call_bytes / (ms_per_step * 1e-3) / 1e9,
                           "frac_measured": call_bytes / (ms_per_step * 1e-3) / 1e9 / peak,

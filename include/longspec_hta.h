@@ -84,7 +84,8 @@ typedef enum {
     /* device-detected, reported by longspec_hta_get_status */
     LONGSPEC_HTA_ERR_BAD_PARENT = -16,         /* some parent[b][i] outside [-1, i) */
     LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE = -17,   /* some prefix_len[b] outside [0, L_cap] */
-    LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT = -18    /* a bounded in-kernel wait ran out */
+    LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT = -18,   /* a bounded in-kernel wait ran out */
+    LONGSPEC_HTA_ERR_INTERNAL = -19            /* a kernel precondition failed (a library bug) */
 } longspec_hta_status;
 
 /* Problem sizes of one call.  scale 0 means 1/sqrt(D); otherwise > 0. */
@@ -99,7 +100,8 @@ typedef struct {
 
 /* Optional knobs of longspec_hta_verify_ex.  Zero-initialise for defaults. */
 typedef struct {
-    int num_splits;          /* prefix split-KV chunks per (b, KV head); 0 = chosen by the library */
+    int num_splits;          /* prefix split-KV chunks per (b, KV head), at most 64 (larger
+                                requests are clamped); 0 = chosen by the library */
     int prefix_kernel;       /* LONGSPEC_HTA_PREFIX_* */
     cudaEvent_t prefix_begin;/* if non-null, recorded on `stream` right before the prefix kernel */
     cudaEvent_t prefix_end;  /* if non-null, recorded on `stream` right after the prefix kernel */

@@ -46,7 +46,7 @@ def test_header_is_plain_c():
 
 def test_abi_version_and_strerror(lib):
     assert lib.longspec_hta_abi_version() == 1
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -16, -17, -18, 12345):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -16, -17, -18, -19, 12345):
         assert lib.longspec_hta_strerror(code)
 
 
@@ -97,6 +97,7 @@ def test_verify_ex_rejects_bad_options(lib):
     (1000, 3, 3, 384),
     (0, 4, 1, 128),
     (262144, 64, 64, 4096),
+    (262144, 100, 64, 4096),
 ])
 def test_chunking_arithmetic(lib, L_cap, req, S, chunk):
     got = hta.chunking(_dims(L_cap=L_cap), req)

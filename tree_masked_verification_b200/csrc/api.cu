@@ -146,7 +146,7 @@ struct Chunking {
 Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms) {
     const int tiles = std::max(1, (d->L_cap + hta::kKeyTile - 1) / hta::kKeyTile);
     auto make = [&](int s) {
-        s = std::max(1, std::min(s, tiles));
+        s = std::max(1, std::min(std::min(s, tiles), hta::kMaxSplits));
         const int ct = (tiles + s - 1) / s;
         return Chunking{(tiles + ct - 1) / ct, ct};
     };
@@ -155,7 +155,7 @@ Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms) {
     const long long units = 1LL * d->B * d->Hkv * m_tiles_of(d);
     Chunking best = make(1);
     double best_cost = 1e300;
-    for (int s = 1; s <= std::min(tiles, 64); ++s) {
+    for (int s = 1; s <= std::min(tiles, hta::kMaxSplits); ++s) {
         const Chunking c = make(s);
         const long long ctas = units * c.S;
         const long long waves = (ctas + num_sms - 1) / std::max(1, num_sms);
@@ -262,6 +262,7 @@ const char *longspec_hta_strerror(int code) {
     case LONGSPEC_HTA_ERR_BAD_PARENT: return "parent[i] outside [-1, i)";
     case LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE: return "prefix_len outside [0, L_cap]";
     case LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT: return "in-kernel wait timed out";
+    case LONGSPEC_HTA_ERR_INTERNAL: return "internal kernel precondition failed";
     default: return "unknown status";
     }
 }
@@ -499,6 +500,7 @@ int longspec_hta_get_status(void *workspace, cudaStream_t stream) {
     if (word & hta::kStatusBadParent) return LONGSPEC_HTA_ERR_BAD_PARENT;
     if (word & hta::kStatusPrefixLenRange) return LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE;
     if (word & hta::kStatusPipelineTimeout) return LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT;
+    if (word & hta::kStatusInternal) return LONGSPEC_HTA_ERR_INTERNAL;
     return LONGSPEC_HTA_OK;
 }
 

@@ -13,6 +13,7 @@ namespace hta {
 
 constexpr int kTreeRowsPerCta = 16;
 constexpr int kKeyTile = 128;   // keys per prefix tile; chunk sizes are multiples of it
+constexpr int kMaxSplits = 64;  // prefix split-KV chunks per (b, KV head), at most
 
 enum TreeMode : int { kTreeModeMerge = 0, kTreeModePartial = 1, kTreeModeMask = 2 };
 

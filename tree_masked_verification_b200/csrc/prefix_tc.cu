@@ -10,25 +10,29 @@
 //
 // CTA = one 128-row tile of the packed query group (rows r = g*T + t of the
 // G query heads sharing KV head kvh) x one KV chunk, so the G*T rows share
-// every K/V tile they read.  Warp roles (320 threads):
-//   warps 0-3  softmax group 0: keys  0..63 of every 128-key tile
-//   warps 4-7  softmax group 1: keys 64..127 of every 128-key tile
+// every K/V tile they read.  Warp roles (384 threads, three warpgroups):
+//   warps 0-3  softmax group 0: P for keys  0..63 of every 128-key tile
+//   warps 4-7  softmax group 1: P for keys 64..127 of every 128-key tile
 //   warp  8    TMA producer: Q once, then K and V tiles into NS-stage rings
 //   warp  9    MMA issuer (one lane) and tensor-memory owner
+//   warps 10-11 idle (complete the third warpgroup)
+// The third warpgroup hands registers to the softmax warpgroups
+// (setmaxnreg): 2 x 128 x 224 + 128 x 56 = 384 x 168, the launch budget.
 // Tensor memory (512 columns x 128 lanes):
 //   S[0], S[1]  cols   0..255  fp32 scores of two tiles in flight; P (bf16
 //                              pairs) is written back over them
 //   O           cols 256..     fp32 output accumulator (D columns)
 //   Q           after O        the Q tile as bf16 pairs (D/2 columns)
-// Q sits in tensor memory so that Q K^T reads only K from shared memory:
-// with both operands in shared memory a 128x128x16 MMA needs the SM's whole
-// shared-memory bandwidth and the tensor pipe starves.
-// Per tile j:  S[j%2] = Q K_j^T (A from tensor memory, B = K), then each
-// softmax group reads its 64 score columns (one row per thread, no
-// shuffles), the two groups exchange their row maxima through shared memory,
-// write P, and O += P V_j (A = P from tensor memory, B = V, N-major).  O is
-// rescaled only when the running max grew by more than 2^8 (a stale max is
-// exact after the final normalisation; P stays <= 256).
+// Q is copied to tensor memory once so that Q K^T reads only K from shared
+// memory (A from tensor memory).
+// Per tile j:  S[j%2] = Q K_j^T (A from tensor memory, B = K); then every
+// softmax thread reads all 128 scores of its row (one row per thread, no
+// shuffles) and takes the row max itself, so both groups reach the same
+// running max with no exchange between them, and each writes P for its 64
+// keys.  Then O += P V_j (A = P from tensor memory, B = V, N-major).  The
+// running max moves only when it grew by more than 2^8 (a stale max is
+// exact after the final normalisation; P stays <= 256); O is rescaled then,
+// each group taking half of its columns.
 #include "hta_kernels.h"
 
 namespace hta {
@@ -49,17 +53,15 @@ struct TcCfg {
     static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
     // barriers: q_full, q_tmem, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    //           s_full[2], p_ready[2], o_ready, o_final, drain
-    static constexpr int NUM_BARS = 2 + 4 * NS + 2 + 2 + 3;
+    //           v_tail, s_full[2], p_ready[2], o_last, o_final, drain
+    static constexpr int NUM_BARS = 2 + 4 * NS + 1 + 2 + 2 + 3;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base (4), abort flag (4)
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;    // slack to align the base to 1024
-    // Once Q is in tensor memory its shared-memory tile is free: the row-max
-    // exchange [parity][group][row] and the epilogue sums [group][2][row]
-    // live there (first written after the first S tile, i.e. after every
-    // warp has finished copying Q).
-    static constexpr int OFF_RED = OFF_Q;
-    static constexpr int OFF_SUMS = OFF_Q + 2 * 2 * 128 * 4;
+    // Once Q is in tensor memory its shared-memory tile is free: the
+    // epilogue's sums [group][2][row] live there (written after the last
+    // P*V, long after every warp has finished copying Q).
+    static constexpr int OFF_SUMS = OFF_Q;
     static constexpr int TMEM_COLS = 512;
     static constexpr int COL_S = 0;                         // S[b] at COL_S + 128*b
     static constexpr int COL_O = 256;
@@ -70,13 +72,17 @@ struct TcCfg {
     static_assert(OFF_SUMS + 2 * 2 * 128 * 4 <= Q_BYTES, "scratch inside the Q tile");
 };
 
-constexpr int kThreadsTc = 320;
+constexpr int kThreadsTc = 384;
+constexpr int kRegsSoftmax = 224;   // per thread, softmax warpgroups
+constexpr int kRegsOther = 56;      // per thread, producer / MMA warpgroup
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreadsTc * 168,
+              "register split must fit the launch allocation");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 
 struct Bars {
-    uint64_t *q_full, *q_tmem, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_ready,
-             *o_ready, *o_final, *drain;
+    uint64_t *q_full, *q_tmem, *k_full, *k_empty, *v_full, *v_empty, *v_tail, *s_full,
+             *p_ready, *o_last, *o_final, *drain;
 };
 
 template <int NS>
@@ -88,10 +94,11 @@ __device__ __forceinline__ Bars carve_bars(uint64_t *base) {
     b.k_empty = b.k_full + NS;
     b.v_full = b.k_empty + NS;
     b.v_empty = b.v_full + NS;
-    b.s_full = b.v_empty + NS;      // [2]
+    b.v_tail = b.v_empty + NS;
+    b.s_full = b.v_tail + 1;        // [2]
     b.p_ready = b.s_full + 2;       // [2]
-    b.o_ready = b.p_ready + 2;
-    b.o_final = b.o_ready + 1;
+    b.o_last = b.p_ready + 2;
+    b.o_final = b.o_last + 1;
     b.drain = b.o_final + 1;
     return b;
 }
@@ -130,6 +137,11 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
+
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
@@ -183,11 +195,12 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(bars.v_full + i, 1);
             mbar_init(bars.v_empty + i, 1);
         }
+        mbar_init(bars.v_tail, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bars.s_full + i, 1);
             mbar_init(bars.p_ready + i, 8);   // one arrive per softmax warp
         }
-        mbar_init(bars.o_ready, 1);
+        mbar_init(bars.o_last, 1);
         mbar_init(bars.o_final, 1);
         mbar_init(bars.drain, 1);
         *s_abort = 0;
@@ -208,6 +221,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     };
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA
+        regs_dec<kRegsOther>();
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -246,87 +260,103 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mbar_wait(bars.v_full + j % C::NS, (j / C::NS) & 1);
             }
         }
+        __syncwarp();
+        if (last_valid < C::BN) {
+            // Keys past L_b may hold anything (even NaN): once the last V tile
+            // has landed, zero its rows past L_b so that P = 0 really adds
+            // nothing, then hand the tile to the MMA warp through v_tail.
+            const int j = n_tiles - 1;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(bars.v_full + j % C::NS, (j / C::NS) & 1));
+            if (ok) {
+                uint8_t *sv = smem + C::OFF_V + (j % C::NS) * C::KV_BYTES;
+                const int per_row = C::HALVES * 8;   // 16-byte chunks per key row
+                for (int idx = lane; idx < (C::BN - last_valid) * per_row; idx += 32) {
+                    const int r = last_valid + idx / per_row;
+                    const int h = (idx % per_row) / 8, c = idx % 8;
+                    *reinterpret_cast<uint4 *>(sv + h * C::BOX_BYTES + r * 128 + c * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.v_tail);
+        }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA
-        bool ok = warp_wait(bars.q_tmem, 0);
-        tc_fence_after();
-        for (int j = 0; ok && j <= n_tiles; ++j) {
-            if (__any_sync(0xffffffffu, *s_abort != 0)) { ok = false; break; }
-            if (j < n_tiles) {
-                // S[j%2] = Q K_j^T : A = Q from tensor memory, B = K (K-major)
-                const int st = j % C::NS;
-                const uint32_t ph = (j / C::NS) & 1;
-                const int sb = j & 1;
-                if (!warp_wait(bars.k_full + st, ph)) { ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t sk = smem_u32(smem + C::OFF_K + st * C::KV_BYTES);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                        mma_ts(tmem + C::COL_S + sb * 128, tmem + C::COL_Q + kk * 8,
-                               smem_desc_sw128(sk + off, 16, 1024), C::IDESC_QK, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bars.k_empty + st);
-                    mma_commit(bars.s_full + sb);
-                }
-                __syncwarp();
-            }
-            if (j >= 1) {
-                // O += P_{j-1} V_{j-1} : A = P from tensor memory, B = V (N-major)
-                const int jj = j - 1;
-                const int st = jj % C::NS;
-                const uint32_t ph = (jj / C::NS) & 1;
-                const int sb = jj & 1;
-                if (!warp_wait(bars.v_full + st, ph)) { ok = false; break; }
-                uint8_t *sv = smem + C::OFF_V + st * C::KV_BYTES;
-                if (jj == n_tiles - 1 && last_valid < C::BN) {
-                    // keys past L_b may hold anything (even NaN): zero their V
-                    // rows so that P = 0 really contributes nothing
-                    const int per_row = C::HALVES * 8;   // 16-byte chunks per key row
-                    for (int idx = lane; idx < (C::BN - last_valid) * per_row; idx += 32) {
-                        const int r = last_valid + idx / per_row;
-                        const int h = (idx % per_row) / 8, c = idx % 8;
-                        *reinterpret_cast<uint4 *>(sv + h * C::BOX_BYTES + r * 128 + c * 16) =
-                            make_uint4(0u, 0u, 0u, 0u);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                if (!warp_wait(bars.p_ready + sb, (jj >> 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t svu = smem_u32(sv);
-#pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk) {
-                        // P of keys 16kk..16kk+15: group kk/4 wrote it at its columns
-                        const uint32_t a = tmem + C::COL_S + sb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-                        const uint64_t bdesc = smem_desc_sw128(svu + kk * 16 * 128, C::BOX_BYTES, 1024);
-                        mma_ts(tmem + C::COL_O, a, bdesc, C::IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(bars.o_ready);
-                    mma_commit(bars.v_empty + st);
-                    if (jj == n_tiles - 1) mma_commit(bars.o_final);
-                }
-                __syncwarp();
-            }
-        }
-        if (!ok) abort_cta();
-        // every MMA this warp issued must be complete before TMEM is freed
+        regs_dec<kRegsOther>();
+        // One thread issues every MMA.  The tensor pipe queues little work,
+        // so each stall of this thread between MMA groups shows up as a pipe
+        // bubble; the loop therefore makes all of a tile's waits at one
+        // point and then issues P*V of tile j-1 and Q K^T of tile j+1 back
+        // to back (16 MMAs).  Order: QK_0, QK_1, [PV_0, QK_2], [PV_1, QK_3],
+        // ...  QK_{j+1} reuses the S buffer of tile j-1, whose P is read by
+        // PV_{j-1} just before it in issue order.
         if (lane == 0) {
+            const uint32_t sk0 = smem_u32(smem + C::OFF_K), sv0 = smem_u32(smem + C::OFF_V);
+            const uint64_t kdesc0 = smem_desc_sw128(sk0, 16, 1024);
+            const uint64_t vdesc0 = smem_desc_sw128(sv0, C::BOX_BYTES, 1024);
+            auto issue_qk = [=](int j) {
+                const int st = j % C::NS, sb = j & 1;
+                const uint64_t kd = kdesc0 + ((st * C::KV_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+                    mma_ts(tmem + C::COL_S + sb * 128, tmem + C::COL_Q + kk * 8, kd + (off >> 4),
+                           C::IDESC_QK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bars.k_empty + st);
+                mma_commit(bars.s_full + sb);
+            };
+            auto issue_pv = [=](int jj) {
+                const int st = jj % C::NS, sb = jj & 1;
+                const uint64_t vd = vdesc0 + ((st * C::KV_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    // P of keys 16kk..16kk+15: group kk/4 wrote it at the start
+                    // of its own 64 score columns
+                    const uint32_t a = tmem + C::COL_S + sb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                    mma_ts(tmem + C::COL_O, a, vd + ((kk * 16 * 128) >> 4), C::IDESC_PV,
+                           (jj > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bars.v_empty + st);
+                if (jj == n_tiles - 2) mma_commit(bars.o_last);
+                if (jj == n_tiles - 1) mma_commit(bars.o_final);
+            };
+            bool ok = mbar_wait(bars.q_tmem, 0);
+            for (int j = 0; ok && j < min(2, n_tiles); ++j) {
+                if (!mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1)) { ok = false; break; }
+                tc_fence_after();
+                issue_qk(j);
+            }
+            for (int jj = 0; ok && jj < n_tiles; ++jj) {
+                const int st = jj % C::NS;
+                const bool tail = (jj == n_tiles - 1) && last_valid < C::BN;
+                const int jn = jj + 2;   // the QK that follows PV_jj in issue order
+                if (!mbar_wait(tail ? bars.v_tail : bars.v_full + st, tail ? 0u : (jj / C::NS) & 1) ||
+                    !mbar_wait(bars.p_ready + (jj & 1), (jj >> 1) & 1) ||
+                    (jn < n_tiles && !mbar_wait(bars.k_full + jn % C::NS, (jn / C::NS) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                issue_pv(jj);
+                if (jn < n_tiles) issue_qk(jn);
+            }
+            if (!ok) abort_cta();
+            // every MMA this thread issued must be complete before TMEM is freed
             mma_commit(bars.drain);
             mbar_wait(bars.drain, 0);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------------- softmax
+        regs_inc<kRegsSoftmax>();
         const int grp = warp >> 2, wq = warp & 3;
         const int r = wq * 32 + lane;                       // row of the tile = TMEM lane
         const bool warp_active = row0 + wq * 32 < p.M;      // any real row in this warp
         const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t t_s = tmem + lane_addr + C::COL_S + grp * 64;
-        const uint32_t t_o = tmem + lane_addr + C::COL_O + grp * (D / 2);
-        float *red = reinterpret_cast<float *>(smem + C::OFF_RED);
+        const uint32_t t_row = tmem + lane_addr + C::COL_S;   // this row's S/P columns
+        const uint32_t t_o = tmem + lane_addr + C::COL_O;     // this row's O columns
         const float c2 = p.scale_log2;
         bool ok = true;
 
@@ -355,60 +385,61 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint64_t l_exact = 0;         // pair of fp32 partial sums of 2^(x - m_run)
         uint64_t l_round = 0;         // the same over the bf16-rounded P that P*V uses
         for (int j = 0; j < n_tiles; ++j) {
-            if (__any_sync(0xffffffffu, *s_abort != 0)) ok = false;
             const int sb = j & 1;
             if (ok && !warp_wait(bars.s_full + sb, (j >> 1) & 1)) { ok = false; abort_cta(); }
             tc_fence_after();
-            const int n_valid = (j == n_tiles - 1) ? last_valid : C::BN;
-            float s[64];
-            float mloc = -INFINITY;
             if (ok && warp_active) {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(t_s + sb * 128, ra);
-                tmem_ld32(t_s + sb * 128 + 32, rb);
+                const int n_valid = (j == n_tiles - 1) ? last_valid : C::BN;
+                // the whole row (128 scores) in one batch of loads
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(t_row + sb * 128 + 0, r0);
+                tmem_ld32(t_row + sb * 128 + 32, r1);
+                tmem_ld32(t_row + sb * 128 + 64, r2);
+                tmem_ld32(t_row + sb * 128 + 96, r3);
                 tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    s[i] = __uint_as_float(ra[i]);
-                    s[32 + i] = __uint_as_float(rb[i]);
-                }
                 if (n_valid < C::BN) {
-                    const int lim = n_valid - grp * 64;
+                    const uint32_t ninf = __float_as_uint(-INFINITY);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) s[i] = (i < lim) ? s[i] : -INFINITY;
+                    for (int i = 0; i < 32; ++i) {
+                        r0[i] = (i < n_valid) ? r0[i] : ninf;
+                        r1[i] = (32 + i < n_valid) ? r1[i] : ninf;
+                        r2[i] = (64 + i < n_valid) ? r2[i] : ninf;
+                        r3[i] = (96 + i < n_valid) ? r3[i] : ninf;
+                    }
                 }
-                float m4[4] = {s[0], s[1], s[2], s[3]};
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int i = 4; i < 64; i += 8) {
-                    m4[0] = max3(m4[0], s[i], s[i + 4]);
-                    m4[1] = max3(m4[1], s[i + 1], s[i + 5]);
-                    m4[2] = max3(m4[2], s[i + 2], s[i + 6]);
-                    m4[3] = max3(m4[3], s[i + 3], s[i + 7]);
+                for (int i = 0; i < 32; i += 2) {
+                    m4[0] = max3(m4[0], __uint_as_float(r0[i]), __uint_as_float(r0[i + 1]));
+                    m4[1] = max3(m4[1], __uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
+                    m4[2] = max3(m4[2], __uint_as_float(r2[i]), __uint_as_float(r2[i + 1]));
+                    m4[3] = max3(m4[3], __uint_as_float(r3[i]), __uint_as_float(r3[i + 1]));
                 }
-                mloc = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
-            }
-            // row max over all 128 keys of the tile: exchange with the other group
-            red[((j & 1) * 2 + grp) * 128 + r] = mloc;
-            named_bar_sync(1, 256);
-            const float mt = fmaxf(red[((j & 1) * 2 + 0) * 128 + r], red[((j & 1) * 2 + 1) * 128 + r]);
-            if (ok && warp_active) {
+                const float mt = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
                 const float m_new = fmaxf(m_run, mt * c2);
                 bool resc = false;
                 float alpha = 1.f;
-                if (m_new > m_run + 8.f) {
-                    alpha = ex2(m_run - m_new);            // 0 on the first tile
-                    l_exact = f2(unf2(l_exact).x * alpha, unf2(l_exact).y * alpha);
-                    l_round = f2(unf2(l_round).x * alpha, unf2(l_round).y * alpha);
+                if (m_new > m_run + 8.f) {                   // lazy update
+                    alpha = ex2(m_run - m_new);              // 0 on the first tile
+                    const uint64_t aa = f2(alpha, alpha);
+                    l_exact = fma2(l_exact, aa, 0ull);
+                    l_round = fma2(l_round, aa, 0ull);
                     resc = j > 0;
                     m_run = m_new;
                 }
                 if (__any_sync(0xffffffffu, resc)) {
-                    // O must hold P*V of tile j-1 before this group rescales its columns
-                    if (!warp_wait(bars.o_ready, (j - 1) & 1)) { ok = false; abort_cta(); }
+                    // O must hold P*V of tile j-1 before this group rescales its
+                    // half of O's columns: S of tile j+1 is committed after that
+                    // P*V was issued, so its completion implies it; the last
+                    // tile has a barrier of its own
+                    const bool done = (j + 1 < n_tiles)
+                        ? warp_wait(bars.s_full + ((j + 1) & 1), ((j + 1) >> 1) & 1)
+                        : warp_wait(bars.o_last, 0);
+                    if (!done) { ok = false; abort_cta(); }
                     tc_fence_after();
                     const float a = resc ? alpha : 1.f;
 #pragma unroll 1
-                    for (int c = 0; c < D / 2; c += 32) {
+                    for (int c = grp * (D / 2); c < (grp + 1) * (D / 2); c += 32) {
                         uint32_t ro[32];
                         tmem_ld32(t_o + c, ro);
                         tmem_wait_ld();
@@ -417,18 +448,26 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         tmem_st32(t_o + c, ro);
                     }
                 }
+                // P for this group's 64 keys, written as bf16 pairs over the
+                // first 32 of its score columns
                 const float mu = (m_run == -INFINITY) ? 0.f : m_run;
                 const uint64_t cc = f2(c2, c2), nm = f2(-mu, -mu);
                 uint32_t pk[32];
+                auto exps = [&](const uint32_t (&ga)[32], const uint32_t (&gb)[32]) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const float2 x = unf2(fma2(f2(s[2 * k], s[2 * k + 1]), cc, nm));
-                    const float p0 = ex2(x.x), p1 = ex2(x.y);
-                    pk[k] = pack_bf16x2(p0, p1);
-                    l_exact = add2(l_exact, f2(p0, p1));
-                    l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
-                }
-                tmem_st32(t_s + sb * 128, pk);
+                    for (int k = 0; k < 32; ++k) {
+                        const uint32_t u0 = (k < 16) ? ga[2 * k] : gb[2 * k - 32];
+                        const uint32_t u1 = (k < 16) ? ga[2 * k + 1] : gb[2 * k + 1 - 32];
+                        const float2 x = unf2(fma2(f2(__uint_as_float(u0), __uint_as_float(u1)), cc, nm));
+                        const float p0 = ex2(x.x), p1 = ex2(x.y);
+                        pk[k] = pack_bf16x2(p0, p1);
+                        l_exact = add2(l_exact, f2(p0, p1));
+                        l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
+                    }
+                };
+                if (grp == 0) exps(r0, r1);
+                else exps(r2, r3);
+                tmem_st32(t_row + sb * 128 + grp * 64, pk);
                 tmem_wait_st();
             }
             tc_fence_before();
@@ -439,6 +478,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ------------------------------------------------------ epilogue
         if (ok && !warp_wait(bars.o_final, 0)) { ok = false; abort_cta(); }
         tc_fence_after();
+        // both groups followed the same running max; add their partial sums
         float *sums = reinterpret_cast<float *>(smem + C::OFF_SUMS);   // [group][exact|round][row]
         const float2 le = unf2(l_exact), lr = unf2(l_round);
         sums[(grp * 2 + 0) * 128 + r] = le.x + le.y;
@@ -450,11 +490,12 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int rr = row0 + r;
         if (warp_active) {
             const float inv = 1.f / l_rd;
+            const uint32_t t_oh = t_o + grp * (D / 2);
             float *dst = p.o_part + ((grow0 + r) * p.S + split) * D + grp * (D / 2);
 #pragma unroll 1
             for (int c = 0; c < D / 2; c += 32) {
                 uint32_t x[32];
-                tmem_ld32(t_o + c, x);
+                tmem_ld32(t_oh + c, x);
                 tmem_wait_ld();
                 if (rr < p.M) {
 #pragma unroll
@@ -471,6 +512,10 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (grp == 0 && rr < p.M)
                 p.lse_part[(grow0 + r) * p.S + split] = failed ? nan : (m_run + lg2(l_ex)) * kLn2;
         }
+    }
+
+    else {
+        regs_dec<kRegsOther>();   // warps 10-11: only complete the warpgroup
     }
 
     tc_fence_before();

@@ -7,6 +7,7 @@
 //
 // One CTA = 8 warps for one (b, KV head) and up to 16 packed rows
 // r = g*T + t of that head's query group.  The CTA
+//   0. stages that head's tree K and V rows in shared memory,
 //   1. loads parent[b][:] into shared memory, checks parent[i] in [-1, i),
 //   2. builds the ancestor-or-self bitmask of every node in shared memory by
 //      pointer jumping (log2 T rounds: anc[i] |= anc[jump[i]],
@@ -33,7 +34,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 template <int D>
 __device__ void tree_rows(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWords],
-                          int b, int kvh, bool bad_parent) {
+                          const __nv_bfloat16 *s_k, const __nv_bfloat16 *s_v, int b, int kvh,
+                          bool bad_parent) {
     constexpr int DPL = D / 32;   // values per lane
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int G = p.Hq / p.Hkv, M = G * p.T, W = (p.T + 31) / 32;
@@ -47,7 +49,6 @@ __device__ void tree_rows(const TreeMergeParams &p, const uint32_t (*anc)[kMaskW
          rr += kWarps) {
         const int g = rr / p.T, t = rr % p.T, h = kvh * G + g;
         const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.T + t;
-        const size_t kv_base = (static_cast<size_t>(b) * p.Hkv + kvh) * p.T;
         float acc[DPL];
         float m = -INFINITY, l = 0.f;
 #pragma unroll
@@ -63,8 +64,8 @@ __device__ void tree_rows(const TreeMergeParams &p, const uint32_t (*anc)[kMaskW
                 while (bits) {
                     const int j = w * 32 + (__ffs(bits) - 1);
                     bits &= bits - 1;
-                    const __nv_bfloat16 *kr = p.k_tree + (kv_base + j) * D + lane * DPL;
-                    const __nv_bfloat16 *vr = p.v_tree + (kv_base + j) * D + lane * DPL;
+                    const __nv_bfloat16 *kr = s_k + j * D + lane * DPL;
+                    const __nv_bfloat16 *vr = s_v + j * D + lane * DPL;
                     float dot = 0.f;
 #pragma unroll
                     for (int i = 0; i < DPL; ++i) dot = fmaf(qv[i], __bfloat162float(kr[i]), dot);
@@ -91,7 +92,7 @@ __device__ void tree_rows(const TreeMergeParams &p, const uint32_t (*anc)[kMaskW
             continue;
         }
 
-        // merge: the tree partial (m, l, acc in log2 units) with S prefix partials
+        // merge: the tree partial (m, l, acc; log2 units) with S prefix partials
         float out_v[DPL];
         float lse_out;
         if (bad_parent || bad_len) {
@@ -101,34 +102,44 @@ __device__ void tree_rows(const TreeMergeParams &p, const uint32_t (*anc)[kMaskW
         } else {
             const float lse2_tree = m + lg2(l);
             const float *lp = p.lse_part + row * p.S;
-            float mx = lse2_tree;
-            bool has_nan = false;
-            for (int s = 0; s < p.S; ++s) {
-                const float v = lp[s];
-                has_nan |= (v != v);
-                mx = fmaxf(mx, v * kLog2e);
-            }
-            float wsum = ex2(lse2_tree - mx);
-            const float wt = wsum / l;
+            // every lane loads up to two partials' lse at once (S <= 64)
+            const float v0 = lane < p.S ? lp[lane] * kLog2e : -INFINITY;
+            const float v1 = lane + 32 < p.S ? lp[lane + 32] * kLog2e : -INFINITY;
+            const bool has_nan = __any_sync(0xffffffffu, (v0 != v0) || (v1 != v1));
+            float mx = fmaxf(fmaxf(v0, v1), lse2_tree);
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) out_v[i] = acc[i] * wt;
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float w0 = ex2(v0 - mx), w1 = ex2(v1 - mx);   // -inf -> 0
+            const float wt = ex2(lse2_tree - mx);
+            const float wsum = warp_sum(w0 + w1) + wt;
+            const float ft = wt / l;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) out_v[i] = acc[i] * ft;
             const float *op = p.o_part + row * static_cast<size_t>(p.S) * D + lane * DPL;
-            for (int s = 0; s < p.S; ++s) {
-                const float v = lp[s];
-                if (v == -INFINITY) continue;
-                const float w = ex2(v * kLog2e - mx);
-                wsum += w;
-                if constexpr (DPL == 4) {
-                    const float4 o4 = *reinterpret_cast<const float4 *>(op + static_cast<size_t>(s) * D);
-                    out_v[0] = fmaf(w, o4.x, out_v[0]);
-                    out_v[1] = fmaf(w, o4.y, out_v[1]);
-                    out_v[2] = fmaf(w, o4.z, out_v[2]);
-                    out_v[3] = fmaf(w, o4.w, out_v[3]);
-                } else {
-                    const float2 o2 = *reinterpret_cast<const float2 *>(op + static_cast<size_t>(s) * D);
-                    out_v[0] = fmaf(w, o2.x, out_v[0]);
-                    out_v[1] = fmaf(w, o2.y, out_v[1]);
+            for (int s0 = 0; s0 < p.S; s0 += 8) {
+                // issue up to 8 partial loads before using any of them
+                float ld[8][DPL];
+                float ws[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int s = s0 + u;
+                    ws[u] = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+                    const bool live = s < p.S && ws[u] > 0.f;
+                    if constexpr (DPL == 4) {
+                        const float4 v = live ? *reinterpret_cast<const float4 *>(op + static_cast<size_t>(s) * D)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                        ld[u][0] = v.x; ld[u][1] = v.y; ld[u][2] = v.z; ld[u][3] = v.w;
+                    } else {
+                        const float2 v = live ? *reinterpret_cast<const float2 *>(op + static_cast<size_t>(s) * D)
+                                              : make_float2(0.f, 0.f);
+                        ld[u][0] = v.x; ld[u][1] = v.y;
+                    }
+                    if (!live) ws[u] = 0.f;
                 }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) out_v[i] = fmaf(ws[u], ld[u][i], out_v[i]);
             }
             const float inv = 1.f / wsum;
 #pragma unroll
@@ -197,7 +208,20 @@ tree_merge_kernel(TreeMergeParams p) {
     __shared__ int s_jump[kTMax];
     __shared__ uint32_t s_anc[kTMax][kMaskWords];
     __shared__ int s_flag;
+    extern __shared__ uint4 s_tree[];   // tree K rows [T][D] then tree V rows [T][D] (bf16)
     const int b = blockIdx.z, kvh = blockIdx.y;
+    if (p.mode != kTreeModeMask) {
+        // stage this head's tree keys and values once (coalesced 16-byte
+        // loads); the __syncthreads of the mask build below orders them
+        const int n16 = p.T * p.D / 8;
+        const size_t base = (static_cast<size_t>(b) * p.Hkv + kvh) * p.T * p.D / 8;
+        const uint4 *kg = reinterpret_cast<const uint4 *>(p.k_tree) + base;
+        const uint4 *vg = reinterpret_cast<const uint4 *>(p.v_tree) + base;
+        for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+            s_tree[i] = kg[i];
+            s_tree[n16 + i] = vg[i];
+        }
+    }
     const bool bad = build_tree_mask(p.parent + static_cast<size_t>(b) * p.T, p.T, s_jump, s_anc, &s_flag);
     if (bad && threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0)
         raise_status(p.status, kStatusBadParent);
@@ -210,19 +234,34 @@ tree_merge_kernel(TreeMergeParams p) {
         }
         return;
     }
-    if (p.D == 128) tree_rows<128>(p, s_anc, b, kvh, bad);
-    else tree_rows<64>(p, s_anc, b, kvh, bad);
+    const __nv_bfloat16 *s_k = reinterpret_cast<const __nv_bfloat16 *>(s_tree);
+    const __nv_bfloat16 *s_v = s_k + p.T * p.D;
+    if (p.D == 128) tree_rows<128>(p, s_anc, s_k, s_v, b, kvh, bad);
+    else tree_rows<64>(p, s_anc, s_k, s_v, b, kvh, bad);
 }
 
 cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream) {
     dim3 grid;
+    size_t smem = 0;
     if (p.mode == kTreeModeMask) {
         grid = dim3(1, 1, p.B);
     } else {
         const int M = (p.Hq / p.Hkv) * p.T;
         grid = dim3((M + kTreeRowsPerCta - 1) / kTreeRowsPerCta, p.Hkv, p.B);
+        smem = static_cast<size_t>(p.T) * p.D * 2 * 2;
+        constexpr int kMaxDev = 64;
+        static bool attr_set[kMaxDev] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (smem > 48 * 1024 && (dev < 0 || dev >= kMaxDev || !attr_set[dev])) {
+            e = cudaFuncSetAttribute(tree_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kTMax) * 128 * 2 * 2);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
+        }
     }
-    tree_merge_kernel<<<grid, kThreads, 0, stream>>>(p);
+    tree_merge_kernel<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -31,6 +31,7 @@ ERR_INVALID_OPTION = -9
 ERR_BAD_PARENT = -16
 ERR_PREFIX_LEN_RANGE = -17
 ERR_PIPELINE_TIMEOUT = -18
+ERR_INTERNAL = -19
 
 PREFIX_TCGEN05 = 0
 PREFIX_SIMT = 1
