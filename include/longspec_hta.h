@@ -161,6 +161,35 @@ LONGSPEC_HTA_API int longspec_hta_verify_ex(const longspec_hta_dims *dims,
                            const longspec_hta_options *opts,
                            cudaStream_t stream);
 
+/*
+ * longspec_hta_verify with no workspace argument, for callers that cannot
+ * allocate device memory (a serving engine that reserves all device memory
+ * at start-up and allows no later allocation, or a decode step in which a
+ * cudaMalloc would synchronise the device).  The pages describe no such
+ * entry point; it has no counterpart there.
+ *   Scratch: a 16 MiB device array inside the library (status word and
+ *   prefix split partials), held by every GPU that loads the library until
+ *   the process exits.  The call picks the largest split count whose
+ *   partials fit; a problem whose partials do not fit even with one split
+ *   (B*Hq*T*(D+1)*4 bytes + 256 > 16 MiB) returns
+ *   LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL and launches nothing.
+ *   Set-up: the first call on each device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.
+ *   Sharing: every call on a device uses the same array.  Calls that can
+ *   overlap on the GPU (different streams, or different host threads with no
+ *   ordering between them) race on it and must be serialised by the caller.
+ *   Device-detected problems (bad parent[], prefix_len out of range) show as
+ *   NaN rows of out/lse; there is no status word to query.
+ *   Allocation: calls no cudaMalloc/cudaFree or any allocating routine.
+ */
+LONGSPEC_HTA_API int longspec_hta_verify_noalloc(const longspec_hta_dims *dims,
+                                const void *q, const void *k_prefix,
+                                const void *v_prefix, const int32_t *prefix_len,
+                                const void *k_tree, const void *v_tree,
+                                const int32_t *parent, void *out, float *lse,
+                                cudaStream_t stream);
+
 /* Device bytes of the staging arena longspec_hta_verify_host needs: room
  * for every input and output plus the workspace, each 256-byte aligned. */
 LONGSPEC_HTA_API size_t longspec_hta_host_arena_bytes(const longspec_hta_dims *dims);

@@ -505,3 +505,79 @@ int longspec_hta_get_status(void *workspace, cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Verification without any device allocation by the caller.
+//
+// Some callers cannot allocate device memory for a workspace: a serving
+// engine that reserves all device memory for its weights and KV cache at
+// start-up and allows no later allocation, or a latency-critical decode
+// step in which a cudaMalloc would synchronise the device.  For them the
+// scratch (status word and prefix split partials) lives in this file-scope
+// device array instead.  Every GPU that loads the library holds it until
+// the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the static scratch on the current device: set up once
+// per device (cudaGetSymbolAddress, a query, not an allocation).  In host
+// code the array's name only stands in for it and must never reach a kernel.
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LONGSPEC_HTA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LONGSPEC_HTA_OK;
+}
+
+}  // namespace
+
+extern "C" int longspec_hta_verify_noalloc(const longspec_hta_dims *dims, const void *q,
+                                           const void *k_prefix, const void *v_prefix,
+                                           const int32_t *prefix_len, const void *k_tree,
+                                           const void *v_tree, const int32_t *parent, void *out,
+                                           float *lse, cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, out, lse};
+    for (const void *p : ptrs) {
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    // the largest split count up to the usual choice whose partials fit
+    int S = chunking_for(dims, 0, di.num_sms).S;
+    while (S > 1 && ws_layout(dims, chunking_for(dims, S, di.num_sms).S).total > kNoAllocScratchBytes) --S;
+    const Chunking c = chunking_for(dims, S, di.num_sms);
+    const WsLayout w = ws_layout(dims, c.S);
+    if (w.total > kNoAllocScratchBytes) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    uint8_t *ws = static_cast<uint8_t *>(scratch);
+    // the array keeps the previous call's contents: the status word must
+    // start at zero; the partials are fully written before they are read
+    if (cudaMemsetAsync(ws, 0, hta::kStatusBytes, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    float *o_part = reinterpret_cast<float *>(ws + w.o_off);
+    float *lse_part = reinterpret_cast<float *>(ws + w.lse_off);
+    const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part, status);
+    if ((rc = run_prefix(dims, pp, LONGSPEC_HTA_PREFIX_TCGEN05, nullptr, nullptr, stream))) return rc;
+    TreeMergeParams tp = tree_params(dims, hta::kTreeModeMerge, c.S, q, k_tree, v_tree, parent,
+                                     prefix_len, o_part, lse_part, status);
+    tp.out = static_cast<__nv_bfloat16 *>(out);
+    tp.lse = lse;
+    return hta::launch_tree_merge(tp, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}

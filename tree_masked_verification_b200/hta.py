@@ -43,7 +43,7 @@ EXPORTED = [
     "longspec_hta_workspace_bytes", "longspec_hta_workspace_init", "longspec_hta_verify",
     "longspec_hta_verify_ex", "longspec_hta_host_arena_bytes", "longspec_hta_verify_host",
     "longspec_hta_tree_mask", "longspec_hta_tree_partial", "longspec_hta_prefix_partial",
-    "longspec_hta_get_status",
+    "longspec_hta_get_status", "longspec_hta_verify_noalloc",
 ]
 
 
