@@ -11,7 +11,7 @@
 
 namespace hta {
 
-constexpr int kTreeRowsPerCta = 16;
+constexpr int kTreeRowsPerCta = 8;    // one warp per packed row
 constexpr int kKeyTile = 128;   // keys per prefix tile; chunk sizes are multiples of it
 constexpr int kMaxSplits = 64;  // prefix split-KV chunks per (b, KV head), at most
 

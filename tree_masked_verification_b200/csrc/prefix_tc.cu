@@ -214,6 +214,8 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    // the tree pass may launch now: it only waits for this grid before merging
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     auto abort_cta = [&]() {
         *s_abort = 1;
