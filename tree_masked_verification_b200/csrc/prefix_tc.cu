@@ -11,28 +11,30 @@
 // CTA = one 128-row tile of the packed query group (rows r = g*T + t of the
 // G query heads sharing KV head kvh) x one KV chunk, so the G*T rows share
 // every K/V tile they read.  Warp roles (384 threads, three warpgroups):
-//   warps 0-3  softmax group 0: P for keys  0..63 of every 128-key tile
-//   warps 4-7  softmax group 1: P for keys 64..127 of every 128-key tile
+//   warps 0-3  softmax group 0: the even key tiles of the chunk
+//   warps 4-7  softmax group 1: the odd key tiles
 //   warp  8    TMA producer: Q once, then K and V tiles into NS-stage rings
 //   warp  9    MMA issuer (one lane) and tensor-memory owner
 //   warps 10-11 idle (complete the third warpgroup)
 // The third warpgroup hands registers to the softmax warpgroups
 // (setmaxnreg): 2 x 128 x 224 + 128 x 56 = 384 x 168, the launch budget.
+// Each group runs its own online softmax (running max m_g, sums l_g) into
+// its own accumulator O_g; the epilogue merges the two exactly, as the lse
+// merge of two KV ranges.  The groups therefore never wait for each other,
+// and the two warps that share an SM sub-partition (w and w+4) work on
+// different tiles, so one of them keeps the exp2 unit busy while the
+// other loads scores and takes its row max.
 // Tensor memory (512 columns x 128 lanes):
-//   S[0], S[1]  cols   0..255  fp32 scores of two tiles in flight; P (bf16
-//                              pairs) is written back over them
-//   O           cols 256..     fp32 output accumulator (D columns)
-//   Q           after O        the Q tile as bf16 pairs (D/2 columns)
-// Q is copied to tensor memory once so that Q K^T reads only K from shared
-// memory (A from tensor memory).
-// Per tile j:  S[j%2] = Q K_j^T (A from tensor memory, B = K); then every
-// softmax thread reads all 128 scores of its row (one row per thread, no
-// shuffles) and takes the row max itself, so both groups reach the same
-// running max with no exchange between them, and each writes P for its 64
-// keys.  Then O += P V_j (A = P from tensor memory, B = V, N-major).  The
-// running max moves only when it grew by more than 2^8 (a stale max is
-// exact after the final normalisation; P stays <= 256); O is rescaled then,
-// each group taking half of its columns.
+//   S[g]   cols 128g..128g+127  fp32 scores of group g's current tile; P
+//                               (bf16 pairs) is written back over them
+//   O[g]   cols 256+gD..        fp32 accumulator of group g (D columns)
+// Per tile j (group g = j%2):  S[g] = Q K_j^T (both operands in shared
+// memory); every thread of group g reads the 128 scores of its row (one row
+// per thread, no shuffles), takes the row max and writes P over the first
+// 64 columns of S[g].  Then O[g] += P V_j (A = P from tensor memory, B = V,
+// N-major).  The running max moves only when it grew by more than 2^8 (a
+// stale max is exact after the final normalisation; P stays <= 256); O[g]
+// is rescaled then.
 #include "hta_kernels.h"
 
 namespace hta {
@@ -52,24 +54,25 @@ struct TcCfg {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-    // barriers: q_full, q_tmem, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    //           v_tail, s_full[2], p_ready[2], o_last, o_final, drain
-    static constexpr int NUM_BARS = 2 + 4 * NS + 1 + 2 + 2 + 3;
+    // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
+    //           v_tail, s_full[2], p_ready[2], o_final, drain
+    static constexpr int NUM_BARS = 1 + 4 * NS + 1 + 2 + 2 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base (4), abort flag (4)
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;    // slack to align the base to 1024
-    // Once Q is in tensor memory its shared-memory tile is free: the
-    // epilogue's sums [group][2][row] live there (written after the last
-    // P*V, long after every warp has finished copying Q).
-    static constexpr int OFF_SUMS = OFF_Q;
+    // After the last MMA the K and V rings are free: the epilogue exchanges
+    // the groups' per-row statistics [group][m|l_exact|l_round][row] in the
+    // first K stage and stages the output rows [row][D] fp32 in the V ring.
+    static constexpr int OFF_XCH = OFF_K;
+    static constexpr int OFF_STAGE = OFF_V;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int COL_S = 0;                         // S[b] at COL_S + 128*b
-    static constexpr int COL_O = 256;
-    static constexpr int COL_Q = COL_O + D;
+    static constexpr int COL_S = 0;                         // S[g] at COL_S + 128*g
+    static constexpr int COL_O = 256;                       // O[g] at COL_O + D*g
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
-    static_assert(COL_Q + D / 2 <= TMEM_COLS, "tensor memory budget");
-    static_assert(OFF_SUMS + 2 * 2 * 128 * 4 <= Q_BYTES, "scratch inside the Q tile");
+    static_assert(COL_O + 2 * D <= TMEM_COLS, "tensor memory budget");
+    static_assert(2 * 3 * 128 * 4 <= KV_BYTES, "statistics exchange inside one K stage");
+    static_assert(BM * D * 4 <= NS * KV_BYTES, "output staging inside the V ring");
 };
 
 constexpr int kThreadsTc = 384;
@@ -81,30 +84,41 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 
 struct Bars {
-    uint64_t *q_full, *q_tmem, *k_full, *k_empty, *v_full, *v_empty, *v_tail, *s_full,
-             *p_ready, *o_last, *o_final, *drain;
+    uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *v_tail, *s_full, *p_ready,
+             *o_final, *drain;
 };
 
 template <int NS>
 __device__ __forceinline__ Bars carve_bars(uint64_t *base) {
     Bars b;
     b.q_full = base;
-    b.q_tmem = base + 1;
-    b.k_full = base + 2;
+    b.k_full = base + 1;
     b.k_empty = b.k_full + NS;
     b.v_full = b.k_empty + NS;
     b.v_empty = b.v_full + NS;
     b.v_tail = b.v_empty + NS;
-    b.s_full = b.v_tail + 1;        // [2]
+    b.s_full = b.v_tail + 1;        // [2], one per group
     b.p_ready = b.s_full + 2;       // [2]
-    b.o_last = b.p_ready + 2;
-    b.o_final = b.o_last + 1;
+    b.o_final = b.p_ready + 2;
     b.drain = b.o_final + 1;
     return b;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// bar.sync over `nthreads` threads that also returns, on every one of them,
+// whether any of them passed `pred` true
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.or.pred q, %1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"(id), "r"(nthreads), "r"(pred ? 1u : 0u) : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -188,7 +202,6 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (threadIdx.x == 0) {
         mbar_init(bars.q_full, 1);
-        mbar_init(bars.q_tmem, 8);
         for (int i = 0; i < C::NS; ++i) {
             mbar_init(bars.k_full + i, 1);
             mbar_init(bars.k_empty + i, 1);
@@ -198,9 +211,8 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(bars.v_tail, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bars.s_full + i, 1);
-            mbar_init(bars.p_ready + i, 8);   // one arrive per softmax warp
+            mbar_init(bars.p_ready + i, 4);   // one arrive per warp of the group
         }
-        mbar_init(bars.o_last, 1);
         mbar_init(bars.o_final, 1);
         mbar_init(bars.drain, 1);
         *s_abort = 0;
@@ -289,42 +301,40 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // One thread issues every MMA.  The tensor pipe queues little work,
         // so each stall of this thread between MMA groups shows up as a pipe
         // bubble; the loop therefore makes all of a tile's waits at one
-        // point and then issues P*V of tile j-1 and Q K^T of tile j+1 back
-        // to back (16 MMAs).  Order: QK_0, QK_1, [PV_0, QK_2], [PV_1, QK_3],
-        // ...  QK_{j+1} reuses the S buffer of tile j-1, whose P is read by
-        // PV_{j-1} just before it in issue order.
+        // point and then issues P*V of tile j and Q K^T of tile j+2 back to
+        // back (16 MMAs).  Order: QK_0, QK_1, [PV_0, QK_2], [PV_1, QK_3], ...
+        // QK_{j+2} reuses S[j%2], whose P is read by PV_j just before it in
+        // issue order (the pipe executes in issue order).
         if (lane == 0) {
+            const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
             const uint32_t sk0 = smem_u32(smem + C::OFF_K), sv0 = smem_u32(smem + C::OFF_V);
             const uint64_t kdesc0 = smem_desc_sw128(sk0, 16, 1024);
             const uint64_t vdesc0 = smem_desc_sw128(sv0, C::BOX_BYTES, 1024);
             auto issue_qk = [=](int j) {
-                const int st = j % C::NS, sb = j & 1;
+                const int st = j % C::NS, g = j & 1;
                 const uint64_t kd = kdesc0 + ((st * C::KV_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                    mma_ts(tmem + C::COL_S + sb * 128, tmem + C::COL_Q + kk * 8, kd + (off >> 4),
+                    mma_ss(tmem + C::COL_S + g * 128, qdesc0 + (off >> 4), kd + (off >> 4),
                            C::IDESC_QK, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bars.k_empty + st);
-                mma_commit(bars.s_full + sb);
+                mma_commit(bars.s_full + g);
             };
             auto issue_pv = [=](int jj) {
-                const int st = jj % C::NS, sb = jj & 1;
+                const int st = jj % C::NS, g = jj & 1;
                 const uint64_t vd = vdesc0 + ((st * C::KV_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    // P of keys 16kk..16kk+15: group kk/4 wrote it at the start
-                    // of its own 64 score columns
-                    const uint32_t a = tmem + C::COL_S + sb * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-                    mma_ts(tmem + C::COL_O, a, vd + ((kk * 16 * 128) >> 4), C::IDESC_PV,
-                           (jj > 0 || kk > 0) ? 1u : 0u);
+                    // P of keys 16kk..16kk+15 sits in columns 8kk..8kk+7 of S[g]
+                    mma_ts(tmem + C::COL_O + g * D, tmem + C::COL_S + g * 128 + kk * 8,
+                           vd + ((kk * 16 * 128) >> 4), C::IDESC_PV, (jj > 1 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bars.v_empty + st);
-                if (jj == n_tiles - 2) mma_commit(bars.o_last);
                 if (jj == n_tiles - 1) mma_commit(bars.o_final);
             };
-            bool ok = mbar_wait(bars.q_tmem, 0);
+            bool ok = mbar_wait(bars.q_full, 0);
             for (int j = 0; ok && j < min(2, n_tiles); ++j) {
                 if (!mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1)) { ok = false; break; }
                 tc_fence_after();
@@ -357,47 +367,25 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int r = wq * 32 + lane;                       // row of the tile = TMEM lane
         const bool warp_active = row0 + wq * 32 < p.M;      // any real row in this warp
         const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t t_row = tmem + lane_addr + C::COL_S;   // this row's S/P columns
-        const uint32_t t_o = tmem + lane_addr + C::COL_O;     // this row's O columns
+        const uint32_t t_s = tmem + lane_addr + C::COL_S + grp * 128;   // this row's S/P
+        const uint32_t t_o = tmem + lane_addr + C::COL_O + grp * D;     // this row's O[grp]
         const float c2 = p.scale_log2;
         bool ok = true;
-
-        // Q tile: shared memory (TMA, 128-byte swizzle) -> tensor memory.
-        // Group g copies the g-th 64-column half of its row.
-        if (!warp_wait(bars.q_full, 0)) { ok = false; abort_cta(); }
-        if (ok && grp < C::HALVES) {
-            const uint8_t *qrow = smem + C::OFF_Q + grp * C::BOX_BYTES + r * 128;
-            uint32_t v[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(qrow + ((c ^ (r & 7)) << 4));
-                v[4 * c + 0] = x.x;
-                v[4 * c + 1] = x.y;
-                v[4 * c + 2] = x.z;
-                v[4 * c + 3] = x.w;
-            }
-            tmem_st32(tmem + lane_addr + C::COL_Q + grp * 32, v);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars.q_tmem);
 
         float m_run = -INFINITY;      // running max of the scaled log2 scores (possibly stale)
         uint64_t l_exact = 0;         // pair of fp32 partial sums of 2^(x - m_run)
         uint64_t l_round = 0;         // the same over the bf16-rounded P that P*V uses
-        for (int j = 0; j < n_tiles; ++j) {
-            const int sb = j & 1;
-            if (ok && !warp_wait(bars.s_full + sb, (j >> 1) & 1)) { ok = false; abort_cta(); }
+        for (int j = grp, it = 0; j < n_tiles; j += 2, ++it) {
+            if (ok && !warp_wait(bars.s_full + grp, it & 1)) { ok = false; abort_cta(); }
             tc_fence_after();
             if (ok && warp_active) {
                 const int n_valid = (j == n_tiles - 1) ? last_valid : C::BN;
                 // the whole row (128 scores) in one batch of loads
                 uint32_t r0[32], r1[32], r2[32], r3[32];
-                tmem_ld32(t_row + sb * 128 + 0, r0);
-                tmem_ld32(t_row + sb * 128 + 32, r1);
-                tmem_ld32(t_row + sb * 128 + 64, r2);
-                tmem_ld32(t_row + sb * 128 + 96, r3);
+                tmem_ld32(t_s + 0, r0);
+                tmem_ld32(t_s + 32, r1);
+                tmem_ld32(t_s + 64, r2);
+                tmem_ld32(t_s + 96, r3);
                 tmem_wait_ld();
                 if (n_valid < C::BN) {
                     const uint32_t ninf = __float_as_uint(-INFINITY);
@@ -422,26 +410,41 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 bool resc = false;
                 float alpha = 1.f;
                 if (m_new > m_run + 8.f) {                   // lazy update
-                    alpha = ex2(m_run - m_new);              // 0 on the first tile
+                    alpha = ex2(m_run - m_new);              // 0 on the group's first tile
                     const uint64_t aa = f2(alpha, alpha);
                     l_exact = fma2(l_exact, aa, 0ull);
                     l_round = fma2(l_round, aa, 0ull);
-                    resc = j > 0;
+                    resc = it > 0;
                     m_run = m_new;
                 }
+                // P for the 128 keys, written as bf16 pairs over the first 64
+                // score columns, 32 scores at a time
+                const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+                const uint64_t cc = f2(c2, c2), nm = f2(-mu, -mu);
+                auto exps = [&](const uint32_t (&sc)[32], int col) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float2 x = unf2(fma2(f2(__uint_as_float(sc[2 * k]), __uint_as_float(sc[2 * k + 1])),
+                                                   cc, nm));
+                        const float p0 = ex2(x.x), p1 = ex2(x.y);
+                        pk[k] = pack_bf16x2(p0, p1);
+                        l_exact = add2(l_exact, f2(p0, p1));
+                        l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
+                    }
+                    tmem_st16(t_s + col, pk);
+                };
+                exps(r0, 0);
+                exps(r1, 16);
+                exps(r2, 32);
+                exps(r3, 48);
                 if (__any_sync(0xffffffffu, resc)) {
-                    // O must hold P*V of tile j-1 before this group rescales its
-                    // half of O's columns: S of tile j+1 is committed after that
-                    // P*V was issued, so its completion implies it; the last
-                    // tile has a barrier of its own
-                    const bool done = (j + 1 < n_tiles)
-                        ? warp_wait(bars.s_full + ((j + 1) & 1), ((j + 1) >> 1) & 1)
-                        : warp_wait(bars.o_last, 0);
-                    if (!done) { ok = false; abort_cta(); }
-                    tc_fence_after();
+                    // S of this tile was committed after P*V of the group's
+                    // previous tile was issued, so O[grp] is complete here, and
+                    // P*V of this tile waits for this warp's arrival below
                     const float a = resc ? alpha : 1.f;
 #pragma unroll 1
-                    for (int c = grp * (D / 2); c < (grp + 1) * (D / 2); c += 32) {
+                    for (int c = 0; c < D; c += 32) {
                         uint32_t ro[32];
                         tmem_ld32(t_o + c, ro);
                         tmem_wait_ld();
@@ -450,70 +453,83 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         tmem_st32(t_o + c, ro);
                     }
                 }
-                // P for this group's 64 keys, written as bf16 pairs over the
-                // first 32 of its score columns
-                const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-                const uint64_t cc = f2(c2, c2), nm = f2(-mu, -mu);
-                uint32_t pk[32];
-                auto exps = [&](const uint32_t (&ga)[32], const uint32_t (&gb)[32]) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const uint32_t u0 = (k < 16) ? ga[2 * k] : gb[2 * k - 32];
-                        const uint32_t u1 = (k < 16) ? ga[2 * k + 1] : gb[2 * k + 1 - 32];
-                        const float2 x = unf2(fma2(f2(__uint_as_float(u0), __uint_as_float(u1)), cc, nm));
-                        const float p0 = ex2(x.x), p1 = ex2(x.y);
-                        pk[k] = pack_bf16x2(p0, p1);
-                        l_exact = add2(l_exact, f2(p0, p1));
-                        l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
-                    }
-                };
-                if (grp == 0) exps(r0, r1);
-                else exps(r2, r3);
-                tmem_st32(t_row + sb * 128 + grp * 64, pk);
                 tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bars.p_ready + sb);
+            if (lane == 0) mbar_arrive(bars.p_ready + grp);
         }
 
         // ------------------------------------------------------ epilogue
         if (ok && !warp_wait(bars.o_final, 0)) { ok = false; abort_cta(); }
         tc_fence_after();
-        // both groups followed the same running max; add their partial sums
-        float *sums = reinterpret_cast<float *>(smem + C::OFF_SUMS);   // [group][exact|round][row]
-        const float2 le = unf2(l_exact), lr = unf2(l_round);
-        sums[(grp * 2 + 0) * 128 + r] = le.x + le.y;
-        sums[(grp * 2 + 1) * 128 + r] = lr.x + lr.y;
-        named_bar_sync(1, 256);
-        const float l_ex = sums[0 * 128 + r] + sums[2 * 128 + r];
-        const float l_rd = sums[1 * 128 + r] + sums[3 * 128 + r];
-        const bool failed = !ok || *s_abort;
+        // merge the two groups' online softmaxes row by row (the lse merge
+        // of two KV ranges): m = max(m_0, m_1), a_g = 2^(m_g - m),
+        // O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1)
+        float *xch = reinterpret_cast<float *>(smem + C::OFF_XCH);   // [grp][m|le|lr][row]
+        {
+            const float2 le = unf2(l_exact), lr = unf2(l_round);
+            xch[(grp * 3 + 0) * 128 + r] = m_run;
+            xch[(grp * 3 + 1) * 128 + r] = le.x + le.y;
+            xch[(grp * 3 + 2) * 128 + r] = lr.x + lr.y;
+        }
+        const bool failed = named_bar_or(1, 256, !ok || *s_abort);
+        const float m0 = xch[0 * 128 + r], m1 = xch[3 * 128 + r];
+        const float m = fmaxf(m0, m1);
+        const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - m);
+        const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - m);   // group 1 had no tile
+        const float l_ex = a0 * xch[1 * 128 + r] + a1 * xch[4 * 128 + r];
+        const float l_rd = a0 * xch[2 * 128 + r] + a1 * xch[5 * 128 + r];
         const int rr = row0 + r;
-        if (warp_active) {
+        if (!failed) {
+            // this group's half of the columns, normalised, into the staging
+            // tile (16-byte chunks of a row XOR-swizzled by row % 8)
             const float inv = 1.f / l_rd;
-            const uint32_t t_oh = t_o + grp * (D / 2);
-            float *dst = p.o_part + ((grow0 + r) * p.S + split) * D + grp * (D / 2);
+            const float c0 = a0 * inv, c1 = a1 * inv;
+            const bool has1 = n_tiles > 1;
+            float *stage = reinterpret_cast<float *>(smem + C::OFF_STAGE);
+            const uint32_t t_o0 = tmem + lane_addr + C::COL_O, t_o1 = t_o0 + D;
+            if (warp_active) {
 #pragma unroll 1
-            for (int c = 0; c < D / 2; c += 32) {
-                uint32_t x[32];
-                tmem_ld32(t_oh + c, x);
-                tmem_wait_ld();
-                if (rr < p.M) {
+                for (int c = grp * (D / 2); c < (grp + 1) * (D / 2); c += 32) {
+                    uint32_t x0[32], x1[32];
+                    tmem_ld32(t_o0 + c, x0);
+                    if (has1) tmem_ld32(t_o1 + c, x1);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
                         float4 v;
-                        v.x = __uint_as_float(x[i + 0]) * inv;
-                        v.y = __uint_as_float(x[i + 1]) * inv;
-                        v.z = __uint_as_float(x[i + 2]) * inv;
-                        v.w = __uint_as_float(x[i + 3]) * inv;
-                        *reinterpret_cast<float4 *>(dst + c + i) = v;
+                        v.x = __uint_as_float(x0[i + 0]) * c0;
+                        v.y = __uint_as_float(x0[i + 1]) * c0;
+                        v.z = __uint_as_float(x0[i + 2]) * c0;
+                        v.w = __uint_as_float(x0[i + 3]) * c0;
+                        if (has1) {
+                            v.x = fmaf(__uint_as_float(x1[i + 0]), c1, v.x);
+                            v.y = fmaf(__uint_as_float(x1[i + 1]), c1, v.y);
+                            v.z = fmaf(__uint_as_float(x1[i + 2]), c1, v.z);
+                            v.w = fmaf(__uint_as_float(x1[i + 3]), c1, v.w);
+                        }
+                        const int q = (c + i) >> 2;          // 16-byte chunk of the row
+                        *reinterpret_cast<float4 *>(stage + r * D + ((q ^ (r & 7)) << 2)) = v;
                     }
                 }
             }
-            if (grp == 0 && rr < p.M)
-                p.lse_part[(grow0 + r) * p.S + split] = failed ? nan : (m_run + lg2(l_ex)) * kLn2;
+            named_bar_sync(1, 256);
+            // coalesced copy-out: a row of o_part is D contiguous floats
+            constexpr int CH = D / 4;                 // chunks per row
+            constexpr int RPI = 32 / CH;              // rows per warp per iteration
+            const int sw = threadIdx.x >> 5;          // softmax warp 0..7
+#pragma unroll 1
+            for (int base = sw * RPI; base < C::BM; base += 8 * RPI) {
+                const int R = base + lane / CH, q = lane % CH;
+                if (row0 + R < p.M) {
+                    const float4 v = *reinterpret_cast<const float4 *>(stage + R * D + ((q ^ (R & 7)) << 2));
+                    *reinterpret_cast<float4 *>(p.o_part + ((grow0 + R) * p.S + split) * D + q * 4) = v;
+                }
+            }
         }
+        if (grp == 0 && warp_active && rr < p.M)
+            p.lse_part[(grow0 + r) * p.S + split] = failed ? nan : (m + lg2(l_ex)) * kLn2;
     }
 
     else {
