@@ -13,9 +13,10 @@
 // every K/V tile they read.  Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax group 0: the even key tiles of the chunk
 //   warps 4-7  softmax group 1: the odd key tiles
-//   warp  8    TMA producer: Q once, then K and V tiles into NS-stage rings
+//   warp  8    TMA producer of Q and the K ring
 //   warp  9    MMA issuer (one lane) and tensor-memory owner
-//   warps 10-11 idle (complete the third warpgroup)
+//   warp  10   TMA producer of the V ring
+//   warp  11   idle (completes the third warpgroup)
 // The third warpgroup hands registers to the softmax warpgroups
 // (setmaxnreg): 2 x 128 x 224 + 128 x 56 = 384 x 168, the launch budget.
 // Each group runs its own online softmax (running max m_g, sums l_g) into
@@ -80,8 +81,9 @@ constexpr int kRegsSoftmax = 224;   // per thread, softmax warpgroups
 constexpr int kRegsOther = 56;      // per thread, producer / MMA warpgroup
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreadsTc * 168,
               "register split must fit the launch allocation");
-constexpr int kProducerWarp = 8;
+constexpr int kProducerKWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kProducerVWarp = 10;
 
 struct Bars {
     uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *v_tail, *s_full, *p_ready,
@@ -233,44 +235,57 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         *s_abort = 1;
         raise_status(p.status, kStatusPipelineTimeout);
     };
-    if (warp == kProducerWarp) {
-        // ------------------------------------------------------------ TMA
+    const int kv_row0 = bk * p.L_cap + key_begin;
+    if (warp == kProducerKWarp) {
+        // -------------------------------------------------------- TMA: Q, K
         regs_dec<kRegsOther>();
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
             uint8_t *sq = smem + C::OFF_Q;
             mbar_arrive_expect_tx(bars.q_full, C::Q_BYTES);
 #pragma unroll
             for (int h = 0; h < C::HALVES; ++h)
                 tma_load_2d(sq + h * C::BOX_BYTES, &tm_q, bars.q_full, h * 64, static_cast<int>(grow0));
-            const int kv_row0 = bk * p.L_cap + key_begin;
-            int k_issued = 0, v_issued = 0;
+            int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % C::NS;
-                const uint32_t ph = (j / C::NS) & 1;
                 if (*s_abort) break;
-                if (!mbar_wait(bars.k_empty + st, ph ^ 1)) { abort_cta(); break; }
+                if (!mbar_wait(bars.k_empty + st, ((j / C::NS) & 1) ^ 1)) { abort_cta(); break; }
                 uint8_t *sk = smem + C::OFF_K + st * C::KV_BYTES;
                 mbar_arrive_expect_tx(bars.k_full + st, C::KV_BYTES);
 #pragma unroll
                 for (int h = 0; h < C::HALVES; ++h)
                     tma_load_2d(sk + h * C::BOX_BYTES, &tm_k, bars.k_full + st, h * 64, kv_row0 + j * C::BN);
-                k_issued = j + 1;
-                if (!mbar_wait(bars.v_empty + st, ph ^ 1)) { abort_cta(); break; }
+                issued = j + 1;
+            }
+            if (*s_abort) {
+                // let the copies in flight land before the CTA releases its smem
+                mbar_wait(bars.q_full, 0);
+                for (int j = max(0, issued - C::NS); j < issued; ++j)
+                    mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kProducerVWarp) {
+        // ----------------------------------------------------------- TMA: V
+        regs_dec<kRegsOther>();
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_v);
+            int issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j % C::NS;
+                if (*s_abort) break;
+                if (!mbar_wait(bars.v_empty + st, ((j / C::NS) & 1) ^ 1)) { abort_cta(); break; }
                 uint8_t *sv = smem + C::OFF_V + st * C::KV_BYTES;
                 mbar_arrive_expect_tx(bars.v_full + st, C::KV_BYTES);
 #pragma unroll
                 for (int h = 0; h < C::HALVES; ++h)
                     tma_load_2d(sv + h * C::BOX_BYTES, &tm_v, bars.v_full + st, h * 64, kv_row0 + j * C::BN);
-                v_issued = j + 1;
+                issued = j + 1;
             }
             if (*s_abort) {
-                // let the copies in flight land before the CTA releases its smem
-                for (int j = max(0, k_issued - C::NS); j < k_issued; ++j)
-                    mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1);
-                for (int j = max(0, v_issued - C::NS); j < v_issued; ++j)
+                for (int j = max(0, issued - C::NS); j < issued; ++j)
                     mbar_wait(bars.v_full + j % C::NS, (j / C::NS) & 1);
             }
         }
@@ -344,9 +359,17 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int st = jj % C::NS;
                 const bool tail = (jj == n_tiles - 1) && last_valid < C::BN;
                 const int jn = jj + 2;   // the QK that follows PV_jj in issue order
-                if (!mbar_wait(tail ? bars.v_tail : bars.v_full + st, tail ? 0u : (jj / C::NS) & 1) ||
-                    !mbar_wait(bars.p_ready + (jj & 1), (jj >> 1) & 1) ||
-                    (jn < n_tiles && !mbar_wait(bars.k_full + jn % C::NS, (jn / C::NS) & 1))) {
+                // the three barriers are probed back to back before any wait
+                uint64_t *bv = tail ? bars.v_tail : bars.v_full + st;
+                const uint32_t pv = tail ? 0u : (jj / C::NS) & 1;
+                uint64_t *bk_ = bars.k_full + (jn < n_tiles ? jn % C::NS : 0);
+                const uint32_t pk = (jn / C::NS) & 1;
+                const bool r1 = mbar_test(smem_u32(bv), pv);
+                const bool r2 = mbar_test(smem_u32(bars.p_ready + (jj & 1)), (jj >> 1) & 1);
+                const bool r3 = jn >= n_tiles || mbar_test(smem_u32(bk_), pk);
+                if (!(r1 && r2 && r3) &&
+                    (!mbar_wait(bv, pv) || !mbar_wait(bars.p_ready + (jj & 1), (jj >> 1) & 1) ||
+                     (jn < n_tiles && !mbar_wait(bk_, pk)))) {
                     ok = false;
                     break;
                 }
@@ -533,7 +556,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 
     else {
-        regs_dec<kRegsOther>();   // warps 10-11: only complete the warpgroup
+        regs_dec<kRegsOther>();   // warp 11: only completes the warpgroup
     }
 
     tc_fence_before();
