@@ -198,6 +198,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const PrefixParams p) {
     using C = TcCfg<D>;
+    // Launched with programmatic stream serialisation: the CTA may be
+    // resident before the previous kernel on the stream has finished, so it
+    // waits for that grid (and its memory) before touching any input.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -618,9 +622,19 @@ cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUte
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
     }
-    dim3 grid(p.m_tiles, p.S, p.B * p.Hkv);
-    prefix_tc_kernel<D><<<grid, kThreadsTc, C::SMEM_ALLOC, stream>>>(tm_q, tm_k, tm_v, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(p.m_tiles, p.S, p.B * p.Hkv);
+    cfg.blockDim = dim3(kThreadsTc);
+    cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+    cfg.stream = stream;
+    // the launch overlaps the tail of the previous kernel on the stream; the
+    // kernel's first instruction waits for that kernel to complete
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefix_tc_kernel<D>, tm_q, tm_k, tm_v, p);
 }
 
 cudaError_t launch_prefix_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,

@@ -124,6 +124,9 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
 
     // merge: the tree partial (m, l, acc; log2 units) with S prefix partials
     grid_dependency_wait();   // the prefix kernel's partials are complete and visible
+    // The next kernel on the stream (the next call's prefix pass) may be
+    // scheduled now: it waits for this grid before it reads anything.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int L = p.prefix_len[b];
     const bool bad_len = L < 0 || L > p.L_cap;
     if (bad_len && lane == 0 && rr == 0) raise_status(p.status, kStatusPrefixLenRange);
