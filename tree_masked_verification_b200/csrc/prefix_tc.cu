@@ -11,13 +11,16 @@
 // CTA = one 128-row tile of the packed query group (rows r = g*T + t of the
 // G query heads sharing KV head kvh) x one KV chunk, so the G*T rows share
 // every K/V tile they read.  Warp roles (384 threads, three warpgroups):
-//   warps 0-3  softmax group 0: the even key tiles of the chunk
-//   warps 4-7  softmax group 1: the odd key tiles
-//   warp  8    TMA producer of Q and the K ring
-//   warp  9    MMA issuer (one lane) and tensor-memory owner
-//   warp  10   TMA producer of the V ring
-//   warp  11   idle (completes the third warpgroup)
-// The third warpgroup hands registers to the softmax warpgroups
+//   warp  0    TMA producer of Q and the K ring
+//   warp  1    MMA issuer (one lane) and tensor-memory owner
+//   warp  2    TMA producer of the V ring
+//   warp  3    idle (completes the first warpgroup)
+//   warps 4-7  softmax group 0: the even key tiles of the chunk
+//   warps 8-11 softmax group 1: the odd key tiles
+// Warp w reaches tensor-memory lanes 32(w%4)..32(w%4)+31 and runs on
+// sub-partition w%4.  The MMA issuer shares its sub-partition with two
+// softmax warps; it has the lower warp index of the three.
+// The first warpgroup hands registers to the softmax warpgroups
 // (setmaxnreg): 2 x 128 x 224 + 128 x 56 = 384 x 168, the launch budget.
 // Each group runs its own online softmax (running max m_g, sums l_g) into
 // its own accumulator O_g; the epilogue merges the two exactly, as the lse
@@ -81,9 +84,10 @@ constexpr int kRegsSoftmax = 224;   // per thread, softmax warpgroups
 constexpr int kRegsOther = 56;      // per thread, producer / MMA warpgroup
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreadsTc * 168,
               "register split must fit the launch allocation");
-constexpr int kProducerKWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kProducerVWarp = 10;
+constexpr int kProducerKWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kProducerVWarp = 2;
+constexpr int kFirstSoftmaxWarp = 4;
 
 struct Bars {
     uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *v_tail, *s_full, *p_ready,
@@ -413,10 +417,10 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_wait(bars.drain, 0);
         }
         __syncwarp();
-    } else if (warp < 8) {
+    } else if (warp >= kFirstSoftmaxWarp) {
         // ------------------------------------------------------- softmax
         regs_inc<kRegsSoftmax>();
-        const int grp = warp >> 2, wq = warp & 3;
+        const int grp = (warp - kFirstSoftmaxWarp) >> 2, wq = warp & 3;
         const int r = wq * 32 + lane;                       // row of the tile = TMEM lane
         const bool warp_active = row0 + wq * 32 < p.M;      // any real row in this warp
         const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
@@ -580,7 +584,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // coalesced copy-out: a row of o_part is D contiguous floats
             constexpr int CH = D / 4;                 // chunks per row
             constexpr int RPI = 32 / CH;              // rows per warp per iteration
-            const int sw = threadIdx.x >> 5;          // softmax warp 0..7
+            const int sw = warp - kFirstSoftmaxWarp;  // softmax warp 0..7
 #pragma unroll 1
             for (int base = sw * RPI; base < C::BM; base += 8 * RPI) {
                 const int R = base + lane / CH, q = lane % CH;
@@ -595,7 +599,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 
     else {
-        regs_dec<kRegsOther>();   // warp 11: only completes the warpgroup
+        regs_dec<kRegsOther>();   // warp 3: only completes the warpgroup
     }
 
     tc_fence_before();
