@@ -85,6 +85,37 @@ def prefix_algorithmic_bytes(w):
     return int(lens.sum()) * w.Hkv * 2 * w.D * 2 + w.B * w.Hq * w.T * w.D * 2
 
 
+def floors(w, peak_gbs):
+    """The three lower bounds of the prefix pass at this pool's peaks (us):
+    HBM (algorithmic bytes / measured copy bandwidth), tensor (the MMA work
+    as issued, 128-row tiles of the G*T packed rows, / measured bf16 cuBLAS
+    throughput; also the useful part alone) and exp2 (one per score / the
+    exp2 unit's 16 results per clock per SM at the maximum SM clock)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        tflops, sm_mhz = float(pk["bf16_tflops"]), float(pk.get("sm_max_mhz", 1965.0))
+    except Exception:
+        tflops, sm_mhz = 1590.0, 1965.0
+    keys = int(w.prefix_lens().astype(np.int64).sum()) * w.Hkv
+    rows = w.G * w.T
+    padded = -(-rows // 128) * 128
+    useful = 4.0 * rows * keys * w.D
+    issued = 4.0 * padded * keys * w.D
+    exps = float(rows * keys)
+    return {"hbm_us": prefix_algorithmic_bytes(w) / (peak_gbs * 1e9) * 1e6,
+            "tensor_us": issued / (tflops * 1e12) * 1e6,
+            "tensor_useful_us": useful / (tflops * 1e12) * 1e6,
+            "exp2_us": exps / (16 * 148 * sm_mhz * 1e6) * 1e6,
+            "basis": f"measured {peak_gbs:.0f} GB/s, {tflops:.0f} TFLOP/s bf16 (burst), "
+                     f"16 exp2/clk/SM x 148 SMs at {sm_mhz:.0f} MHz"}
+
+
+def pct(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))]
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -303,19 +334,33 @@ def run_ours(args, world, rank, local):
     # around the prefix kernel on the launching stream
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    for a, b in ev:          # torch creates the CUDA event on first record
+    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for (a, b), c in zip(ev, ev_end):   # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
+        c.record(stream)
     barrier(world)
     torch.cuda.synchronize()
     for i in range(args.steps):
         call(i, ev[i])
+        ev_end[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     prefix_ms = [a.elapsed_time(b) for a, b in ev]
+    call_ms = [a.elapsed_time(c) for (a, _), c in zip(ev, ev_end)]
     prefix_avg_ms = max_over_ranks(sum(prefix_ms) / len(prefix_ms), world)
     if hta.get_status(ws) != hta.OK:
         raise RuntimeError("device status error in the roofline region")
+
+    # host cost of one call (argument checks, tensor-map lookup, launches),
+    # the GPU running behind it
+    torch.cuda.synchronize()
+    n_host = min(args.steps, 100)
+    h0 = time.perf_counter()
+    for i in range(n_host):
+        call(i)
+    host_us = (time.perf_counter() - h0) / n_host * 1e6
+    torch.cuda.synchronize()
 
     ms_per_step = elapsed_ms / args.steps
     us_per_call = job_us_per_call(elapsed_ms, args.steps, world)
@@ -342,6 +387,15 @@ def run_ours(args, world, rank, local):
         "call_roofline": {"bytes": call_bytes, "achieved_gbs": call_bytes / (ms_per_step * 1e-3) / 1e9,
                           "frac_measured": call_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
                           "frac_nominal_8tbs": call_bytes / (ms_per_step * 1e-3) / 8e12},
+        "distribution": {
+            "call_us": {"p10": pct(call_ms, 0.1) * 1e3, "p50": pct(call_ms, 0.5) * 1e3,
+                        "p90": pct(call_ms, 0.9) * 1e3},
+            "prefix_us": {"p10": pct(prefix_ms, 0.1) * 1e3, "p50": pct(prefix_ms, 0.5) * 1e3,
+                          "p90": pct(prefix_ms, 0.9) * 1e3},
+            "host_api_us_per_call": host_us,
+            "note": "per-call CUDA events of the roofline pass (events between the kernels "
+                    "serialise them, so these run a little above the headline value)"},
+        "floors": floors(w, peak),
         "gpu_launches": 2 * args.steps,
         "timing": "value: CUDA events around the K back-to-back calls; roofline: a second pass "
                   "of the same calls with events around each prefix launch",

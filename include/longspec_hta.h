@@ -253,6 +253,19 @@ LONGSPEC_HTA_API int longspec_hta_prefix_partial(const longspec_hta_dims *dims, 
  * and returns LONGSPEC_HTA_OK or the first device-detected error. */
 LONGSPEC_HTA_API int longspec_hta_get_status(void *workspace, cudaStream_t stream);
 
+/* Self-test of failure detection (a test hook; the pages define no such
+ * operation).  Launches one CTA on `stream` whose thread waits, with the
+ * same bounded wait as every pipeline stage of the verification kernels,
+ * on a barrier that nothing completes.  After the bound (about 2 s of SM
+ * cycles) the wait gives up and sets the PIPELINE_TIMEOUT bit in the
+ * status word of `workspace` (device memory, 16-byte aligned, at least
+ * 256 bytes, e.g. a verification workspace), exactly as a stalled stage
+ * would; the kernel then returns and the context stays usable.  Returns
+ * LONGSPEC_HTA_OK once launched, NULL_POINTER / MISALIGNED /
+ * UNSUPPORTED_DEVICE / CUDA otherwise; longspec_hta_get_status then
+ * reports LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT. */
+LONGSPEC_HTA_API int longspec_hta_selftest_wait_timeout(void *workspace, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -490,6 +490,16 @@ int longspec_hta_prefix_partial(const longspec_hta_dims *dims, const void *q, co
     return run_prefix(dims, pp, prefix_kernel, nullptr, nullptr, stream);
 }
 
+int longspec_hta_selftest_wait_timeout(void *workspace, cudaStream_t stream) {
+    if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    if (!aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    DeviceInfo dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return hta::launch_wait_timeout_selftest(static_cast<uint32_t *>(workspace), stream) == cudaSuccess
+               ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
 int longspec_hta_get_status(void *workspace, cudaStream_t stream) {
     if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;

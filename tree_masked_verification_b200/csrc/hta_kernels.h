@@ -46,6 +46,8 @@ struct PrefixParams {
 };
 
 cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream);
+// One bounded wait that is left to run out; sets kStatusPipelineTimeout.
+cudaError_t launch_wait_timeout_selftest(uint32_t *status, cudaStream_t stream);
 cudaError_t launch_prefix_simt(const PrefixParams &p, cudaStream_t stream);
 // Tensor maps: q as [B*Hq*T][D], k/v as [B*Hkv*L_cap][D], box 64 x 128, 128B swizzle.
 cudaError_t launch_prefix_tc(const PrefixParams &p, const CUtensorMap &tm_q,

@@ -44,6 +44,7 @@ EXPORTED = [
     "longspec_hta_verify_ex", "longspec_hta_host_arena_bytes", "longspec_hta_verify_host",
     "longspec_hta_tree_mask", "longspec_hta_tree_partial", "longspec_hta_prefix_partial",
     "longspec_hta_get_status", "longspec_hta_verify_noalloc",
+    "longspec_hta_selftest_wait_timeout",
 ]
 
 
@@ -98,6 +99,7 @@ def load():
             lib.longspec_hta_prefix_partial.argtypes = [pd, vp, vp, vp, vp, vp, vp, ci, ci,
                                                         ctypes.POINTER(ci), vp, sz, vp]
             lib.longspec_hta_get_status.argtypes = [vp, vp]
+            lib.longspec_hta_selftest_wait_timeout.argtypes = [vp, vp]
             lib.longspec_hta_chunking.argtypes = [pd, ci, ctypes.POINTER(ci), ctypes.POINTER(ci)]
             _lib = lib
     return _lib
@@ -264,6 +266,13 @@ def prefix_partial(q, k_prefix, v_prefix, prefix_len, *, scale: float = 0.0,
     if S_out.value != S:
         raise RuntimeError(f"split count mismatch: library {S_out.value}, binding {S}")
     return o, l, chunk_keys
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, stream=None) -> int:
+    """Launch the failure-detection self-test on `workspace`'s status word:
+    one bounded in-kernel wait that nothing completes (about 2 s); a later
+    get_status() returns ERR_PIPELINE_TIMEOUT."""
+    return int(load().longspec_hta_selftest_wait_timeout(_ptr(workspace), _stream(stream)))
 
 
 def get_status(workspace: torch.Tensor, stream=None) -> int:
