@@ -139,6 +139,24 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
     } else {
         const float lse2_tree = m + lg2(l);
         const float *lp = p.lse_part + row * p.S;
+        const float *op = p.o_part + row * static_cast<size_t>(p.S) * D + lane * DPL;
+        // the lse of every partial and the first 8 partial rows are loaded in
+        // one round: the O loads do not wait for the weights (a partial with
+        // weight 0 is dropped by a select below, so a slot a chunk past L_b
+        // never wrote cannot leak in, whatever it holds)
+        float ld[8][DPL];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if constexpr (DPL == 4) {
+                const float4 v = u < p.S ? *reinterpret_cast<const float4 *>(op + static_cast<size_t>(u) * D)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                ld[u][0] = v.x; ld[u][1] = v.y; ld[u][2] = v.z; ld[u][3] = v.w;
+            } else {
+                const float2 v = u < p.S ? *reinterpret_cast<const float2 *>(op + static_cast<size_t>(u) * D)
+                                         : make_float2(0.f, 0.f);
+                ld[u][0] = v.x; ld[u][1] = v.y;
+            }
+        }
         // every lane loads up to two partials' lse at once (S <= 64)
         const float v0 = lane < p.S ? lp[lane] * kLog2e : -INFINITY;
         const float v1 = lane + 32 < p.S ? lp[lane + 32] * kLog2e : -INFINITY;
@@ -155,31 +173,30 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
         const float ft = wt / l;
 #pragma unroll
         for (int i = 0; i < DPL; ++i) out_v[i] = acc[i] * ft;
-        const float *op = p.o_part + row * static_cast<size_t>(p.S) * D + lane * DPL;
         for (int s0 = 0; s0 < p.S; s0 += 8) {
-            // issue up to 8 partial loads before using any of them
-            float ld[8][DPL];
-            float ws[8];
+            if (s0 > 0) {   // partials 8.. (more than 8 splits): one more round per 8
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int s = s0 + u;
+                    if constexpr (DPL == 4) {
+                        const float4 v = s < p.S ? *reinterpret_cast<const float4 *>(op + static_cast<size_t>(s) * D)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                        ld[u][0] = v.x; ld[u][1] = v.y; ld[u][2] = v.z; ld[u][3] = v.w;
+                    } else {
+                        const float2 v = s < p.S ? *reinterpret_cast<const float2 *>(op + static_cast<size_t>(s) * D)
+                                                 : make_float2(0.f, 0.f);
+                        ld[u][0] = v.x; ld[u][1] = v.y;
+                    }
+                }
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int s = s0 + u;
-                ws[u] = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-                const bool use = s < p.S && ws[u] > 0.f;
-                if constexpr (DPL == 4) {
-                    const float4 v = use ? *reinterpret_cast<const float4 *>(op + static_cast<size_t>(s) * D)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                    ld[u][0] = v.x; ld[u][1] = v.y; ld[u][2] = v.z; ld[u][3] = v.w;
-                } else {
-                    const float2 v = use ? *reinterpret_cast<const float2 *>(op + static_cast<size_t>(s) * D)
-                                         : make_float2(0.f, 0.f);
-                    ld[u][0] = v.x; ld[u][1] = v.y;
-                }
-                if (!use) ws[u] = 0.f;
+                const float ws = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+                const bool use = s < p.S && ws > 0.f;
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) out_v[i] = use ? fmaf(ws, ld[u][i], out_v[i]) : out_v[i];
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                for (int i = 0; i < DPL; ++i) out_v[i] = fmaf(ws[u], ld[u][i], out_v[i]);
         }
         const float inv = 1.f / wsum;
 #pragma unroll
