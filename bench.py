@@ -117,8 +117,9 @@ def pct(xs, q):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms; only the
+    samples stamped inside the timed region are kept."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -135,7 +136,10 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t_begin=None, t_end=None):
+        """Median SM clock and throttle reasons of the samples taken between
+        the host wall times t_begin and t_end (all samples if none fall in)."""
+        import datetime
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -144,23 +148,25 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in out.splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]),
+                             {n for n, v in zip(names, f[6:10]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        inside = [r for r in rows if t_begin is not None and t_begin - 0.05 <= r[0] <= t_end + 0.05]
+        use = inside or rows
+        if not use:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "samples": len(sm),
+        reasons = set().union(*(r[3] for r in use))
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": use[-1][2],
+                "samples": len(use), "samples_in_timed_region": len(inside),
                 "reasons": sorted(reasons)}
 
 
@@ -254,8 +260,13 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     total_rows = w.B * w.Hq * w.T
-    per_step = max(1, min(w.G * w.T, args.ref_rows))
     heads = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    # a step is a bounded sample of the call: as many query rows as keep the
+    # whole run within --ref-budget seconds (at least one row, at most
+    # --ref-rows), from the time of one row measured first
+    spent1, _ = oracle_rows_timed(w, heads[:1], 0.0, rows_per_head=1)
+    fit = int(args.ref_budget / max(1, args.warmup + args.steps) / max(spent1, 1e-9))
+    per_step = max(1, min(w.G * w.T, args.ref_rows, fit))
     times = []
     for i in range(args.warmup + args.steps):
         spent, rows = oracle_rows_timed(w, heads[:1], 0.0, rows_per_head=per_step,
@@ -319,29 +330,32 @@ def run_ours(args, world, rank, local):
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    wall0 = time.time()
     t_start.record(stream)
     for i in range(args.steps):
         call(i)
     t_end.record(stream)
     torch.cuda.synchronize()
+    wall1 = time.time()
     barrier(world)
-    clocks = sampler.stop()
+    clocks = sampler.stop(wall0, wall1)
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     if hta.get_status(ws) != hta.OK:
         raise RuntimeError("device status error in the timed region")
 
     # timed region 2 (the roofline): the same calls with CUDA events recorded
     # around the prefix kernel on the launching stream
+    n2 = min(args.steps, 2000)   # calls of the second pass (per-call events)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+          for _ in range(n2)]
+    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(n2)]
     for (a, b), c in zip(ev, ev_end):   # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
         c.record(stream)
     barrier(world)
     torch.cuda.synchronize()
-    for i in range(args.steps):
+    for i in range(n2):
         call(i, ev[i])
         ev_end[i].record(stream)
     torch.cuda.synchronize()
@@ -440,7 +454,7 @@ def run_e2e(args, w, cpu, dims, dev, stream, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3-8b-32k", choices=sorted(WORKLOADS))
@@ -448,6 +462,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
