@@ -51,8 +51,11 @@ def peaks():
 
 def workload_config(w, S, n_sets):
     tree = {"levels": "/".join(map(str, w.widths)), "random": "random", "chain": "chain"}[w.tree]
+    if w.kind == "prefix":
+        tree = "none (prefix-only attention)"
     lens = w.prefix_lens()
-    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "T": w.T,
+    return {"workload": w.name, "call": "longspec_hta_prefix_attention" if w.kind == "prefix"
+            else "longspec_hta_verify", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "T": w.T,
             "L_cap": w.L_cap, "L_mean": float(lens.mean()), "tree": tree,
             "k_peaked": w.k_peaked, "num_splits": S,
             "l2": f"inputs rotate over {n_sets} buffer sets ({n_sets}x the K/V bytes > 2x L2)"
@@ -237,7 +240,10 @@ def oracle_rows_timed(w, heads, budget_s, rows_per_head=None, row_offset=0):
         rows = np.array([[0, ((row_offset + r) % M) // w.T, ((row_offset + r) % M) % w.T]
                          for r in range(n)], dtype=np.int32)
         t0 = time.perf_counter()
-        p.attention(rows)
+        if w.kind == "prefix":
+            p.prefix_partial(0, w.L_cap, rows)
+        else:
+            p.attention(rows)
         spent += time.perf_counter() - t0
         done += n
         if spent >= budget_s:
@@ -311,9 +317,14 @@ def run_ours(args, world, rank, local):
 
     def call(i, events=None):
         s = sets[i % n_sets]
-        hta.verify(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], s["k_tree"],
-                   s["v_tree"], s["parent"], out=out, lse=lse, workspace=ws, scale=w.scale,
-                   num_splits=args.num_splits, prefix_events=events, stream=stream)
+        if w.kind == "prefix":
+            hta.prefix_attention(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], out=out,
+                                 lse=lse, workspace=ws, scale=w.scale, num_splits=args.num_splits,
+                                 prefix_events=events, stream=stream)
+        else:
+            hta.verify(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], s["k_tree"],
+                       s["v_tree"], s["parent"], out=out, lse=lse, workspace=ws, scale=w.scale,
+                       num_splits=args.num_splits, prefix_events=events, stream=stream)
 
     for i in range(args.warmup):
         call(i)
@@ -392,7 +403,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": us_per_call, "unit": "µs", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, 4/16/16/16/16 tree)",
+        "data": f"synthetic (seeded N(0,1) bf16; tree: {workload_config(w, S, n_sets)['tree']})",
         "config": workload_config(w, S, n_sets),
         "roofline": {"bound": "hbm", "kernel": "prefix_tc_kernel", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
@@ -422,15 +433,35 @@ def run_ours(args, world, rank, local):
 
 
 def run_e2e(args, w, cpu, dims, dev, stream, world):
-    host = {k: v.pin_memory() for k, v in cpu.items()}
-    arena = torch.empty(hta.host_arena_bytes(dims), dtype=torch.uint8, device=dev)
+    names = (("q", "k_prefix", "v_prefix", "prefix_len") if w.kind == "prefix"
+             else tuple(cpu.keys()))
+    host = {k: cpu[k].pin_memory() for k in names}
     out = torch.empty_like(host["q"]).pin_memory()
     lse = torch.empty(host["q"].shape[:3], dtype=torch.float32).pin_memory()
+    if w.kind == "prefix":
+        # no host-buffer entry point for prefix-only attention: the same
+        # copies in and out around the device call, all on `stream`
+        dsts = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        dout = torch.empty_like(dsts["q"])
+        dlse = torch.empty(dsts["q"].shape[:3], dtype=torch.float32, device=dev)
+        ws = hta.new_workspace(dims, args.num_splits, dev)
 
-    def call():
-        hta.verify_host(host["q"], host["k_prefix"], host["v_prefix"], host["prefix_len"],
-                        host["k_tree"], host["v_tree"], host["parent"], out, lse, arena,
-                        scale=w.scale, stream=stream)
+        def call():
+            with torch.cuda.stream(stream):
+                for k, v in host.items():
+                    dsts[k].copy_(v, non_blocking=True)
+                hta.prefix_attention(dsts["q"], dsts["k_prefix"], dsts["v_prefix"],
+                                     dsts["prefix_len"], out=dout, lse=dlse, workspace=ws,
+                                     scale=w.scale, num_splits=args.num_splits, stream=stream)
+                out.copy_(dout, non_blocking=True)
+                lse.copy_(dlse, non_blocking=True)
+    else:
+        arena = torch.empty(hta.host_arena_bytes(dims), dtype=torch.uint8, device=dev)
+
+        def call():
+            hta.verify_host(host["q"], host["k_prefix"], host["v_prefix"], host["prefix_len"],
+                            host["k_tree"], host["v_tree"], host["parent"], out, lse, arena,
+                            scale=w.scale, stream=stream)
 
     steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(min(args.warmup, 3)):

@@ -249,6 +249,24 @@ LONGSPEC_HTA_API int longspec_hta_prefix_partial(const longspec_hta_dims *dims, 
                                 void *workspace, size_t workspace_bytes,
                                 cudaStream_t stream);
 
+/* Attention of the query rows to the prefix alone: no tree keys, no mask.
+ * This is the draft model's cross-attention into the target's KV cache in
+ * LongSpec (LongSpec paper summary, "Summary": the draft attends to the
+ * target model's KV cache), the prefix pass of verify followed by the same
+ * exact lse merge of its split-KV partials, without the tree partial:
+ *   out[b][h][t] = sum_{j < L_b} e^{s q.k_j - m} v_j / sum_{j < L_b} e^{s q.k_j - m},
+ *   lse[b][h][t] = m + ln sum_{j < L_b} e^{s q.k_j - m}   (natural log).
+ * dims->T is the number of query tokens per head (1 <= T <= 256); q, k_prefix,
+ * v_prefix, prefix_len, out and lse have the layouts of longspec_hta_verify;
+ * there is no k_tree, v_tree or parent.  A row with L_b = 0 sees no key:
+ * its out is 0 and its lse is -inf.  workspace / options / errors: as
+ * longspec_hta_verify_ex (longspec_hta_workspace_bytes gives the size). */
+LONGSPEC_HTA_API int longspec_hta_prefix_attention(const longspec_hta_dims *dims, const void *q,
+                                  const void *k_prefix, const void *v_prefix,
+                                  const int32_t *prefix_len, void *out, float *lse,
+                                  void *workspace, size_t workspace_bytes,
+                                  const longspec_hta_options *opts, cudaStream_t stream);
+
 /* Synchronises `stream`, reads and clears the status word of `workspace`,
  * and returns LONGSPEC_HTA_OK or the first device-detected error. */
 LONGSPEC_HTA_API int longspec_hta_get_status(void *workspace, cudaStream_t stream);

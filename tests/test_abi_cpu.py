@@ -112,3 +112,28 @@ def test_workspace_bytes_formula(lib):
     rows = 1 * 32 * 68
     assert n >= 256 + rows * 6 * 129 * 4
     assert n - (256 + rows * 6 * 129 * 4) < 1024
+
+
+def test_prefix_attention_rejects_bad_arguments_on_host(lib):
+    """Prefix-only attention: q, k_prefix, v_prefix, prefix_len, out, lse and
+    the workspace are checked (NULL, 16-byte alignment, dims, options)
+    before any device work."""
+    d = _dims()
+    ptrs = [4096 * (i + 1) for i in range(6)]
+    ws = 4096 * 20
+    for i in range(6):
+        bad = list(ptrs)
+        bad[i] = 0
+        assert lib.longspec_hta_prefix_attention(ctypes.byref(d), *bad, ws, 1 << 30, None,
+                                                 None) == hta.ERR_NULL_POINTER
+        bad[i] = ptrs[i] + 8
+        assert lib.longspec_hta_prefix_attention(ctypes.byref(d), *bad, ws, 1 << 30, None,
+                                                 None) == hta.ERR_MISALIGNED
+    assert lib.longspec_hta_prefix_attention(ctypes.byref(d), *ptrs, 0, 1 << 30, None,
+                                             None) == hta.ERR_NULL_POINTER
+    bad_dims = _dims(D=96)
+    assert lib.longspec_hta_prefix_attention(ctypes.byref(bad_dims), *ptrs, ws, 1 << 30, None,
+                                             None) != hta.OK
+    opts = hta.Options(-1, 0, None, None)
+    assert lib.longspec_hta_prefix_attention(ctypes.byref(d), *ptrs, ws, 1 << 30, ctypes.byref(opts),
+                                             None) == hta.ERR_INVALID_OPTION

@@ -490,6 +490,41 @@ int longspec_hta_prefix_partial(const longspec_hta_dims *dims, const void *q, co
     return run_prefix(dims, pp, prefix_kernel, nullptr, nullptr, stream);
 }
 
+int longspec_hta_prefix_attention(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                                  const void *v_prefix, const int32_t *prefix_len, void *out, float *lse,
+                                  void *workspace, size_t workspace_bytes,
+                                  const longspec_hta_options *opts, cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, out, lse, workspace};
+    for (const void *p : ptrs) {
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    longspec_hta_options o{};
+    if (opts) o = *opts;
+    if (o.num_splits < 0 || (o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
+                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
+        return LONGSPEC_HTA_ERR_INVALID_OPTION;
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms);
+    const WsLayout w = ws_layout(dims, c.S);
+    if (workspace_bytes < w.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    float *o_part = reinterpret_cast<float *>(ws + w.o_off);
+    float *lse_part = reinterpret_cast<float *>(ws + w.lse_off);
+
+    const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part, status);
+    if ((rc = run_prefix(dims, pp, o.prefix_kernel, o.prefix_begin, o.prefix_end, stream))) return rc;
+    TreeMergeParams tp = tree_params(dims, hta::kTreeModePrefixOnly, c.S, q, nullptr, nullptr, nullptr,
+                                     prefix_len, o_part, lse_part, status);
+    tp.out = static_cast<__nv_bfloat16 *>(out);
+    tp.lse = lse;
+    return hta::launch_tree_merge(tp, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
 int longspec_hta_selftest_wait_timeout(void *workspace, cudaStream_t stream) {
     if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
     if (!aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;

@@ -15,7 +15,11 @@ constexpr int kTreeRowsPerCta = 8;    // one warp per packed row
 constexpr int kKeyTile = 128;   // keys per prefix tile; chunk sizes are multiples of it
 constexpr int kMaxSplits = 64;  // prefix split-KV chunks per (b, KV head), at most
 
-enum TreeMode : int { kTreeModeMerge = 0, kTreeModePartial = 1, kTreeModeMask = 2 };
+// Merge: tree pass + lse merge with the prefix partials.  PrefixOnly: the
+// merge of the prefix partials alone (no tree keys; q rows attend to the
+// prefix only).  Partial / Mask: debug exports of the tree pass.
+enum TreeMode : int { kTreeModeMerge = 0, kTreeModePartial = 1, kTreeModeMask = 2,
+                      kTreeModePrefixOnly = 3 };
 
 struct TreeMergeParams {
     int B, Hq, Hkv, D, T, L_cap, S;

@@ -47,7 +47,7 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
 
-    if (!bad_parent) {
+    if (!bad_parent && p.mode != kTreeModePrefixOnly) {
         float qv[DPL];
         const __nv_bfloat16 *qr = p.q + row * D + lane * DPL;
 #pragma unroll
@@ -170,7 +170,7 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
         wsum += wt;
-        const float ft = wt / l;
+        const float ft = l > 0.f ? wt / l : 0.f;   // no tree keys: weight 0
 #pragma unroll
         for (int i = 0; i < DPL; ++i) out_v[i] = acc[i] * ft;
         for (int s0 = 0; s0 < p.S; s0 += 8) {
@@ -199,9 +199,10 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
             }
         }
         const float inv = 1.f / wsum;
+        const bool empty = mx == -INFINITY;   // no visible key at all (prefix-only, L_b = 0)
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) out_v[i] = has_nan ? nan : out_v[i] * inv;
-        lse_out = has_nan ? nan : (mx + lg2(wsum)) * kLn2;
+        for (int i = 0; i < DPL; ++i) out_v[i] = has_nan ? nan : empty ? 0.f : out_v[i] * inv;
+        lse_out = has_nan ? nan : empty ? -INFINITY : (mx + lg2(wsum)) * kLn2;
     }
     __nv_bfloat16 *orow = p.out + row * D + lane * DPL;
     if constexpr (DPL == 4) {
@@ -265,7 +266,10 @@ tree_merge_kernel(TreeMergeParams p) {
     __shared__ uint32_t s_anc[kTMax][kMaskWords];
     __shared__ int s_flag;
     const int b = blockIdx.z, kvh = blockIdx.y;
-    const bool bad = build_tree_mask(p.parent + static_cast<size_t>(b) * p.T, p.T, s_jump, s_anc, &s_flag);
+    // no tree keys in the prefix-only merge: no parent array, no mask
+    const bool bad = p.mode == kTreeModePrefixOnly
+                         ? false
+                         : build_tree_mask(p.parent + static_cast<size_t>(b) * p.T, p.T, s_jump, s_anc, &s_flag);
     if (bad && threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0)
         raise_status(p.status, kStatusBadParent);
 
@@ -295,7 +299,7 @@ cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream) {
         const int M = (p.Hq / p.Hkv) * p.T;
         cfg.gridDim = dim3((M + kTreeRowsPerCta - 1) / kTreeRowsPerCta, p.Hkv, p.B);
     }
-    if (p.mode == kTreeModeMerge) {
+    if (p.mode == kTreeModeMerge || p.mode == kTreeModePrefixOnly) {
         // may start while the prefix kernel finishes; the merge waits for it
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;

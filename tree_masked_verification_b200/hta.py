@@ -44,7 +44,7 @@ EXPORTED = [
     "longspec_hta_verify_ex", "longspec_hta_host_arena_bytes", "longspec_hta_verify_host",
     "longspec_hta_tree_mask", "longspec_hta_tree_partial", "longspec_hta_prefix_partial",
     "longspec_hta_get_status", "longspec_hta_verify_noalloc",
-    "longspec_hta_selftest_wait_timeout",
+    "longspec_hta_selftest_wait_timeout", "longspec_hta_prefix_attention",
 ]
 
 
@@ -91,6 +91,7 @@ def load():
             lib.longspec_hta_workspace_init.argtypes = [vp, sz, vp]
             lib.longspec_hta_verify.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
             lib.longspec_hta_verify_ex.argtypes = [pd] + [vp] * 9 + [vp, sz, ctypes.POINTER(Options), vp]
+            lib.longspec_hta_prefix_attention.argtypes = [pd] + [vp] * 6 + [vp, sz, ctypes.POINTER(Options), vp]
             lib.longspec_hta_host_arena_bytes.argtypes = [pd]
             lib.longspec_hta_host_arena_bytes.restype = sz
             lib.longspec_hta_verify_host.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
@@ -188,6 +189,35 @@ def verify(q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, *, out=Non
         ctypes.byref(dims), _ptr(q), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_len),
         _ptr(k_tree), _ptr(v_tree), _ptr(parent), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), ctypes.byref(opts), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def prefix_attention(q, k_prefix, v_prefix, prefix_len, *, out=None, lse=None, workspace=None,
+                     scale: float = 0.0, num_splits: int = 0, prefix_kernel: int = PREFIX_TCGEN05,
+                     prefix_events=None, stream=None):
+    """Attention of q's rows to the prefix alone (no tree keys, no mask):
+    the draft model's cross-attention into the target's KV cache.  q is
+    [B][Hq][T][D] with T query tokens per head.  Returns (out bf16, lse fp32);
+    rows of a sequence with L_b = 0 get out 0 and lse -inf."""
+    dev = q.device
+    for t, n in ((q, "q"), (k_prefix, "k_prefix"), (v_prefix, "v_prefix")):
+        _need(t, n, torch.bfloat16, dev)
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    dims = dims_of(q, k_prefix, scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(dims, num_splits, dev)
+    opts = Options(int(num_splits), int(prefix_kernel),
+                   prefix_events[0].cuda_event if prefix_events else None,
+                   prefix_events[1].cuda_event if prefix_events else None)
+    rc = load().longspec_hta_prefix_attention(
+        ctypes.byref(dims), _ptr(q), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_len),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        ctypes.byref(opts), _stream(stream))
     _check(rc)
     return out, lse
 

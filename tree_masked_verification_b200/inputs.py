@@ -97,6 +97,10 @@ class Workload:
     prefix_range: Optional[Tuple[int, int]] = None   # None -> every L_b = L_cap
     k_peaked: bool = False
     scale: float = 0.0                        # 0 -> 1/sqrt(D)
+    # "verify": prefix + tree (longspec_hta_verify); "prefix": the T query
+    # tokens attend to the prefix alone (longspec_hta_prefix_attention, the
+    # draft model's cross-attention into the target's KV cache)
+    kind: str = "verify"
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -214,6 +218,8 @@ class Workload:
         out = self.B * self.Hq * self.T * self.D * 2
         lse = self.B * self.Hq * self.T * 4
         idx = self.B * self.T * 4 + self.B * 4
+        if self.kind == "prefix":   # no tree K/V, no parent array
+            return kv + q + out + lse + self.B * 4
         return kv + q + tree + out + lse + idx
 
 
@@ -235,4 +241,9 @@ WORKLOADS = {
     "ultra-256k-chain5": Workload("ultra-256k-chain5", B=1, Hq=32, Hkv=8,
                                   D=128, T=5, L_cap=262144, seed=5,
                                   tree="chain"),
+    # the draft model's cross-attention into the Llama-3-8B target's KV
+    # cache: 4 draft tokens per head, no tree keys
+    "draft-xattn-32k": Workload("draft-xattn-32k", B=1, Hq=32, Hkv=8, D=128,
+                                T=4, L_cap=32768, seed=6, tree="chain",
+                                kind="prefix"),
 }
