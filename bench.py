@@ -32,7 +32,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from tree_masked_verification_b200 import hta  # noqa: E402
-from tree_masked_verification_b200.inputs import WORKLOADS  # noqa: E402
+from tree_masked_verification_b200.inputs import WORKLOADS, paged_cache  # noqa: E402
 
 METRIC = "µs per layer verify-attention call; achieved HBM GB/s vs B200 peak @32k prefix"
 L2_BYTES = 126 * 1024 * 1024
@@ -54,8 +54,11 @@ def workload_config(w, S, n_sets):
     if w.kind == "prefix":
         tree = "none (prefix-only attention)"
     lens = w.prefix_lens()
-    return {"workload": w.name, "call": "longspec_hta_prefix_attention" if w.kind == "prefix"
-            else "longspec_hta_verify", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "T": w.T,
+    call = "longspec_hta_prefix_attention" if w.kind == "prefix" else "longspec_hta_verify"
+    if w.block_size:
+        call += "_paged"
+    return {"workload": w.name, "call": call, "block_size": w.block_size or None,
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "T": w.T,
             "L_cap": w.L_cap, "L_mean": float(lens.mean()), "tree": tree,
             "k_peaked": w.k_peaked, "num_splits": S,
             "l2": f"inputs rotate over {n_sets} buffer sets ({n_sets}x the K/V bytes > 2x L2)"
@@ -300,8 +303,13 @@ def run_reference(args, world, rank):
 # --------------------------------------------------------------------------
 def run_ours(args, world, rank, local):
     w = WORKLOADS[args.workload]
+    if args.block_size >= 0:
+        w = w.replace(block_size=args.block_size)
     dev = torch.device("cuda", torch.cuda.current_device())
     cpu = w.generate()
+    if w.block_size:
+        cpu["k_cache"], cpu["v_cache"], cpu["block_table"] = paged_cache(
+            cpu["k_prefix"], cpu["v_prefix"], cpu["prefix_len"].tolist(), w.block_size, w.seed)
     kv_bytes = 2 * cpu["k_prefix"].numel() * 2
     n_sets = 1 if kv_bytes > 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / kv_bytes)) + 1
     sets = []
@@ -317,7 +325,13 @@ def run_ours(args, world, rank, local):
 
     def call(i, events=None):
         s = sets[i % n_sets]
-        if w.kind == "prefix":
+        if w.block_size:
+            fn = hta.prefix_attention_paged if w.kind == "prefix" else hta.verify_paged
+            tree = () if w.kind == "prefix" else (s["k_tree"], s["v_tree"], s["parent"])
+            fn(s["q"], s["k_cache"], s["v_cache"], s["block_table"], s["prefix_len"], *tree,
+               L_cap=w.L_cap, out=out, lse=lse, workspace=ws, scale=w.scale,
+               num_splits=args.num_splits, prefix_events=events, stream=stream)
+        elif w.kind == "prefix":
             hta.prefix_attention(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], out=out,
                                  lse=lse, workspace=ws, scale=w.scale, num_splits=args.num_splits,
                                  prefix_events=events, stream=stream)
@@ -433,26 +447,42 @@ def run_ours(args, world, rank, local):
 
 
 def run_e2e(args, w, cpu, dims, dev, stream, world):
-    names = (("q", "k_prefix", "v_prefix", "prefix_len") if w.kind == "prefix"
-             else tuple(cpu.keys()))
+    if w.block_size:
+        names = ("q", "k_cache", "v_cache", "block_table", "prefix_len") + (
+            () if w.kind == "prefix" else ("k_tree", "v_tree", "parent"))
+    elif w.kind == "prefix":
+        names = ("q", "k_prefix", "v_prefix", "prefix_len")
+    else:
+        names = tuple(cpu.keys())
     host = {k: cpu[k].pin_memory() for k in names}
     out = torch.empty_like(host["q"]).pin_memory()
     lse = torch.empty(host["q"].shape[:3], dtype=torch.float32).pin_memory()
-    if w.kind == "prefix":
-        # no host-buffer entry point for prefix-only attention: the same
-        # copies in and out around the device call, all on `stream`
+    if w.kind == "prefix" or w.block_size:
+        # no host-buffer entry point for these calls: the same copies in and
+        # out around the device call, all on `stream`
         dsts = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
         dout = torch.empty_like(dsts["q"])
         dlse = torch.empty(dsts["q"].shape[:3], dtype=torch.float32, device=dev)
         ws = hta.new_workspace(dims, args.num_splits, dev)
 
+        def device_call():
+            s = dsts
+            if w.block_size:
+                fn = hta.prefix_attention_paged if w.kind == "prefix" else hta.verify_paged
+                tree = () if w.kind == "prefix" else (s["k_tree"], s["v_tree"], s["parent"])
+                fn(s["q"], s["k_cache"], s["v_cache"], s["block_table"], s["prefix_len"], *tree,
+                   L_cap=w.L_cap, out=dout, lse=dlse, workspace=ws, scale=w.scale,
+                   num_splits=args.num_splits, stream=stream)
+            else:
+                hta.prefix_attention(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], out=dout,
+                                     lse=dlse, workspace=ws, scale=w.scale,
+                                     num_splits=args.num_splits, stream=stream)
+
         def call():
             with torch.cuda.stream(stream):
                 for k, v in host.items():
                     dsts[k].copy_(v, non_blocking=True)
-                hta.prefix_attention(dsts["q"], dsts["k_prefix"], dsts["v_prefix"],
-                                     dsts["prefix_len"], out=dout, lse=dlse, workspace=ws,
-                                     scale=w.scale, num_splits=args.num_splits, stream=stream)
+                device_call()
                 out.copy_(dout, non_blocking=True)
                 lse.copy_(dlse, non_blocking=True)
     else:
@@ -490,6 +520,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3-8b-32k", choices=sorted(WORKLOADS))
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--block-size", type=int, default=-1,
+                    help="paged prefix cache block size for the workload (0 = contiguous; "
+                         "default: the workload's own)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=16)

@@ -85,7 +85,8 @@ typedef enum {
     LONGSPEC_HTA_ERR_BAD_PARENT = -16,         /* some parent[b][i] outside [-1, i) */
     LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE = -17,   /* some prefix_len[b] outside [0, L_cap] */
     LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT = -18,   /* a bounded in-kernel wait ran out */
-    LONGSPEC_HTA_ERR_INTERNAL = -19            /* a kernel precondition failed (a library bug) */
+    LONGSPEC_HTA_ERR_INTERNAL = -19,           /* a kernel precondition failed (a library bug) */
+    LONGSPEC_HTA_ERR_BAD_BLOCK = -20           /* a block_table entry outside [0, num_blocks) */
 } longspec_hta_status;
 
 /* Problem sizes of one call.  scale 0 means 1/sqrt(D); otherwise > 0. */
@@ -106,6 +107,28 @@ typedef struct {
     cudaEvent_t prefix_begin;/* if non-null, recorded on `stream` right before the prefix kernel */
     cudaEvent_t prefix_end;  /* if non-null, recorded on `stream` right after the prefix kernel */
 } longspec_hta_options;
+
+/* A paged prefix KV cache (the block-table layout of serving engines): the
+ * keys of sequence b are cut into blocks of block_size consecutive
+ * positions; block_table[b][i] names the cache block that holds positions
+ * [i*block_size, (i+1)*block_size) of sequence b for every KV head.
+ *   k_cache, v_cache: bf16 [num_blocks][Hkv][block_size][D], device, 16-byte
+ *                     aligned; block n, KV head h, position p at
+ *                     ((n*Hkv + h)*block_size + p)*D.
+ *   block_table:      int32 [B][max_blocks], device; entries past the last
+ *                     block a sequence uses are not read.
+ *   block_size:       16, 32, 64 or 128.
+ *   max_blocks:       >= ceil(L_cap / block_size).
+ * An entry outside [0, num_blocks) is read as block 0 and reported by
+ * longspec_hta_get_status as LONGSPEC_HTA_ERR_BAD_BLOCK. */
+typedef struct {
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_table;
+    int num_blocks;
+    int block_size;
+    int max_blocks;
+} longspec_hta_paged_kv;
 
 /* ABI version of the loaded library (LONGSPEC_HTA_ABI_VERSION). */
 LONGSPEC_HTA_API int longspec_hta_abi_version(void);
@@ -266,6 +289,26 @@ LONGSPEC_HTA_API int longspec_hta_prefix_attention(const longspec_hta_dims *dims
                                   const int32_t *prefix_len, void *out, float *lse,
                                   void *workspace, size_t workspace_bytes,
                                   const longspec_hta_options *opts, cudaStream_t stream);
+
+/* longspec_hta_verify_ex and longspec_hta_prefix_attention with the prefix
+ * K/V read from a paged cache (longspec_hta_paged_kv) instead of the
+ * contiguous [B][Hkv][L_cap][D] arrays; every other argument, the result
+ * and the error behaviour are the same.  The results equal those of the
+ * contiguous call on the same keys bit for bit (same kernels, same split).
+ * Only the tcgen05 prefix kernel reads a paged cache: prefix_kernel
+ * LONGSPEC_HTA_PREFIX_SIMT returns LONGSPEC_HTA_ERR_INVALID_OPTION.  Host
+ * errors: NULL_POINTER / MISALIGNED for the cache and table pointers,
+ * INVALID_DIMS for a block_size not in {16, 32, 64, 128}, num_blocks < 1,
+ * max_blocks * block_size < L_cap or a cache over 2^31 rows. */
+LONGSPEC_HTA_API int longspec_hta_verify_paged(const longspec_hta_dims *dims, const void *q,
+                                const longspec_hta_paged_kv *kv, const int32_t *prefix_len,
+                                const void *k_tree, const void *v_tree, const int32_t *parent,
+                                void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                const longspec_hta_options *opts, cudaStream_t stream);
+LONGSPEC_HTA_API int longspec_hta_prefix_attention_paged(const longspec_hta_dims *dims, const void *q,
+                                const longspec_hta_paged_kv *kv, const int32_t *prefix_len,
+                                void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                const longspec_hta_options *opts, cudaStream_t stream);
 
 /* Synchronises `stream`, reads and clears the status word of `workspace`,
  * and returns LONGSPEC_HTA_OK or the first device-detected error. */

@@ -137,3 +137,30 @@ def test_prefix_attention_rejects_bad_arguments_on_host(lib):
     opts = hta.Options(-1, 0, None, None)
     assert lib.longspec_hta_prefix_attention(ctypes.byref(d), *ptrs, ws, 1 << 30, ctypes.byref(opts),
                                              None) == hta.ERR_INVALID_OPTION
+
+
+def test_paged_calls_reject_bad_arguments_on_host(lib):
+    """Paged cache descriptor checks: NULL descriptor or table, block sizes
+    outside {16, 32, 64, 128}, a table too short for L_cap, and the SIMT
+    prefix kernel (which reads contiguous K/V only)."""
+    d = _dims(L_cap=1024)
+    base = dict(k_cache=4096 * 30, v_cache=4096 * 31, block_table=4096 * 32, num_blocks=64,
+                block_size=16, max_blocks=64)
+
+    def call(kv, opts=None):
+        ptrs = [4096 * (i + 1) for i in range(6)]   # q, prefix_len, k_tree, v_tree, parent, out
+        return lib.longspec_hta_verify_paged(ctypes.byref(d), ptrs[0],
+                                             None if kv is None else ctypes.byref(kv), *ptrs[1:],
+                                             4096 * 20, 4096 * 21, 1 << 30,
+                                             None if opts is None else ctypes.byref(opts), None)
+
+    assert call(None) == hta.ERR_NULL_POINTER
+    assert call(hta.PagedKV(**{**base, "block_table": 0})) == hta.ERR_NULL_POINTER
+    assert call(hta.PagedKV(**{**base, "k_cache": 0})) == hta.ERR_NULL_POINTER
+    assert call(hta.PagedKV(**{**base, "v_cache": base["v_cache"] + 8})) == hta.ERR_MISALIGNED
+    for bs in (8, 24, 256):
+        assert call(hta.PagedKV(**{**base, "block_size": bs})) == hta.ERR_INVALID_DIMS
+    assert call(hta.PagedKV(**{**base, "max_blocks": 63})) == hta.ERR_INVALID_DIMS
+    assert call(hta.PagedKV(**{**base, "num_blocks": 0})) == hta.ERR_INVALID_DIMS
+    simt = hta.Options(0, hta.PREFIX_SIMT, None, None)
+    assert call(hta.PagedKV(**base), simt) == hta.ERR_INVALID_OPTION

@@ -70,8 +70,9 @@ struct MapKey {
     const void *ptr;
     uint64_t rows;
     int D;
+    int box_rows;
     bool operator==(const MapKey &o) const {
-        return dev == o.dev && ptr == o.ptr && rows == o.rows && D == o.D;
+        return dev == o.dev && ptr == o.ptr && rows == o.rows && D == o.D && box_rows == o.box_rows;
     }
 };
 struct MapEntry {
@@ -84,11 +85,13 @@ MapEntry g_maps[kMapCache];
 int g_map_next = 0;
 std::mutex g_map_mu;
 
-// [rows][D] bf16 matrix as 64-column x 128-row boxes with 128-byte swizzle.
-int tensor_map(const void *ptr, uint64_t rows, int D, CUtensorMap *out) {
+// [rows][D] bf16 matrix as 64-column x box_rows-row boxes with 128-byte
+// swizzle (box_rows 128 for Q and contiguous K/V, the block size for a
+// paged cache).
+int tensor_map(const void *ptr, uint64_t rows, int D, CUtensorMap *out, int box_rows = 128) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
-    const MapKey key{dev, ptr, rows, D};
+    const MapKey key{dev, ptr, rows, D, box_rows};
     std::lock_guard<std::mutex> lk(g_map_mu);
     for (auto &e : g_maps)
         if (e.used && e.key == key) { *out = e.map; return LONGSPEC_HTA_OK; }
@@ -97,7 +100,7 @@ int tensor_map(const void *ptr, uint64_t rows, int D, CUtensorMap *out) {
     CUtensorMap m;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -206,11 +209,14 @@ int run_prefix(const longspec_hta_dims *d, const PrefixParams &p, int kernel, cu
     CUtensorMap tq, tk, tv;
     if (kernel == LONGSPEC_HTA_PREFIX_TCGEN05) {
         const uint64_t qrows = 1ull * d->B * d->Hq * d->T;
-        const uint64_t krows = 1ull * d->B * d->Hkv * std::max(d->L_cap, 1);
+        const bool paged = p.block_table != nullptr;
+        const uint64_t krows = paged ? 1ull * p.num_blocks * d->Hkv * p.block_size
+                                     : 1ull * d->B * d->Hkv * std::max(d->L_cap, 1);
+        const int box = paged ? p.block_size : 128;
         int rc;
         if ((rc = tensor_map(p.q, qrows, d->D, &tq)) != LONGSPEC_HTA_OK) return rc;
-        if ((rc = tensor_map(p.k_prefix, krows, d->D, &tk)) != LONGSPEC_HTA_OK) return rc;
-        if ((rc = tensor_map(p.v_prefix, krows, d->D, &tv)) != LONGSPEC_HTA_OK) return rc;
+        if ((rc = tensor_map(p.k_prefix, krows, d->D, &tk, box)) != LONGSPEC_HTA_OK) return rc;
+        if ((rc = tensor_map(p.v_prefix, krows, d->D, &tv, box)) != LONGSPEC_HTA_OK) return rc;
     }
     if (ev_begin && cudaEventRecord(ev_begin, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
     cudaError_t e = (kernel == LONGSPEC_HTA_PREFIX_TCGEN05)
@@ -263,6 +269,7 @@ const char *longspec_hta_strerror(int code) {
     case LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE: return "prefix_len outside [0, L_cap]";
     case LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT: return "in-kernel wait timed out";
     case LONGSPEC_HTA_ERR_INTERNAL: return "internal kernel precondition failed";
+    case LONGSPEC_HTA_ERR_BAD_BLOCK: return "a block_table entry is outside [0, num_blocks)";
     default: return "unknown status";
     }
 }
@@ -312,22 +319,40 @@ int longspec_hta_workspace_init(void *workspace, size_t workspace_bytes, cudaStr
                                                                                   : LONGSPEC_HTA_ERR_CUDA;
 }
 
-int longspec_hta_verify_ex(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
-                           const void *v_prefix, const int32_t *prefix_len, const void *k_tree,
-                           const void *v_tree, const int32_t *parent, void *out, float *lse,
-                           void *workspace, size_t workspace_bytes,
-                           const longspec_hta_options *opts, cudaStream_t stream) {
+// One verification call (prefix_only = false) or prefix-only attention
+// (prefix_only = true), the prefix K/V contiguous (kv == nullptr) or paged.
+static int run_attention(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                         const void *v_prefix, const longspec_hta_paged_kv *kv,
+                         const int32_t *prefix_len, const void *k_tree, const void *v_tree,
+                         const int32_t *parent, void *out, float *lse, void *workspace,
+                         size_t workspace_bytes, const longspec_hta_options *opts,
+                         cudaStream_t stream, bool prefix_only) {
     int rc = check_dims(dims);
     if (rc) return rc;
-    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, k_tree, v_tree, parent, out, lse, workspace};
+    if (kv) {
+        k_prefix = kv->k_cache;
+        v_prefix = kv->v_cache;
+        if (!kv->block_table) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if ((reinterpret_cast<uintptr_t>(kv->block_table) & 3u) != 0) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, out, lse, workspace,
+                          prefix_only ? q : k_tree, prefix_only ? q : v_tree, prefix_only ? q : parent};
     for (const void *p : ptrs) {
         if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
         if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
     }
+    if (kv) {
+        const int bs = kv->block_size;
+        if ((bs != 16 && bs != 32 && bs != 64 && bs != 128) || kv->num_blocks < 1 || kv->max_blocks < 1 ||
+            1LL * kv->max_blocks * bs < dims->L_cap ||
+            1LL * kv->num_blocks * dims->Hkv * bs + 128 >= (1LL << 31))
+            return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    }
     longspec_hta_options o{};
     if (opts) o = *opts;
     if (o.num_splits < 0 || (o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
-                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
+                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT) ||
+        (kv && o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05))
         return LONGSPEC_HTA_ERR_INVALID_OPTION;
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
@@ -339,13 +364,41 @@ int longspec_hta_verify_ex(const longspec_hta_dims *dims, const void *q, const v
     float *o_part = reinterpret_cast<float *>(ws + w.o_off);
     float *lse_part = reinterpret_cast<float *>(ws + w.lse_off);
 
-    const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part, status);
+    PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part, status);
+    if (kv) {
+        pp.block_table = kv->block_table;
+        pp.block_size = kv->block_size;
+        pp.max_blocks = kv->max_blocks;
+        pp.num_blocks = kv->num_blocks;
+    }
     if ((rc = run_prefix(dims, pp, o.prefix_kernel, o.prefix_begin, o.prefix_end, stream))) return rc;
-    TreeMergeParams tp = tree_params(dims, hta::kTreeModeMerge, c.S, q, k_tree, v_tree, parent,
-                                     prefix_len, o_part, lse_part, status);
+    TreeMergeParams tp = prefix_only
+        ? tree_params(dims, hta::kTreeModePrefixOnly, c.S, q, nullptr, nullptr, nullptr, prefix_len,
+                      o_part, lse_part, status)
+        : tree_params(dims, hta::kTreeModeMerge, c.S, q, k_tree, v_tree, parent, prefix_len, o_part,
+                      lse_part, status);
     tp.out = static_cast<__nv_bfloat16 *>(out);
     tp.lse = lse;
     return hta::launch_tree_merge(tp, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
+int longspec_hta_verify_ex(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
+                           const void *v_prefix, const int32_t *prefix_len, const void *k_tree,
+                           const void *v_tree, const int32_t *parent, void *out, float *lse,
+                           void *workspace, size_t workspace_bytes,
+                           const longspec_hta_options *opts, cudaStream_t stream) {
+    return run_attention(dims, q, k_prefix, v_prefix, nullptr, prefix_len, k_tree, v_tree, parent, out,
+                         lse, workspace, workspace_bytes, opts, stream, false);
+}
+
+int longspec_hta_verify_paged(const longspec_hta_dims *dims, const void *q, const longspec_hta_paged_kv *kv,
+                              const int32_t *prefix_len, const void *k_tree, const void *v_tree,
+                              const int32_t *parent, void *out, float *lse, void *workspace,
+                              size_t workspace_bytes, const longspec_hta_options *opts,
+                              cudaStream_t stream) {
+    if (!kv) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    return run_attention(dims, q, nullptr, nullptr, kv, prefix_len, k_tree, v_tree, parent, out, lse,
+                         workspace, workspace_bytes, opts, stream, false);
 }
 
 int longspec_hta_verify(const longspec_hta_dims *dims, const void *q, const void *k_prefix,
@@ -494,35 +547,17 @@ int longspec_hta_prefix_attention(const longspec_hta_dims *dims, const void *q, 
                                   const void *v_prefix, const int32_t *prefix_len, void *out, float *lse,
                                   void *workspace, size_t workspace_bytes,
                                   const longspec_hta_options *opts, cudaStream_t stream) {
-    int rc = check_dims(dims);
-    if (rc) return rc;
-    const void *ptrs[] = {q, k_prefix, v_prefix, prefix_len, out, lse, workspace};
-    for (const void *p : ptrs) {
-        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
-        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
-    }
-    longspec_hta_options o{};
-    if (opts) o = *opts;
-    if (o.num_splits < 0 || (o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
-                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
-        return LONGSPEC_HTA_ERR_INVALID_OPTION;
-    DeviceInfo di;
-    if ((rc = current_device(&di))) return rc;
-    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms);
-    const WsLayout w = ws_layout(dims, c.S);
-    if (workspace_bytes < w.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
-    float *o_part = reinterpret_cast<float *>(ws + w.o_off);
-    float *lse_part = reinterpret_cast<float *>(ws + w.lse_off);
+    return run_attention(dims, q, k_prefix, v_prefix, nullptr, prefix_len, nullptr, nullptr, nullptr, out,
+                         lse, workspace, workspace_bytes, opts, stream, true);
+}
 
-    const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part, status);
-    if ((rc = run_prefix(dims, pp, o.prefix_kernel, o.prefix_begin, o.prefix_end, stream))) return rc;
-    TreeMergeParams tp = tree_params(dims, hta::kTreeModePrefixOnly, c.S, q, nullptr, nullptr, nullptr,
-                                     prefix_len, o_part, lse_part, status);
-    tp.out = static_cast<__nv_bfloat16 *>(out);
-    tp.lse = lse;
-    return hta::launch_tree_merge(tp, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+int longspec_hta_prefix_attention_paged(const longspec_hta_dims *dims, const void *q,
+                                        const longspec_hta_paged_kv *kv, const int32_t *prefix_len,
+                                        void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                        const longspec_hta_options *opts, cudaStream_t stream) {
+    if (!kv) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    return run_attention(dims, q, nullptr, nullptr, kv, prefix_len, nullptr, nullptr, nullptr, out, lse,
+                         workspace, workspace_bytes, opts, stream, true);
 }
 
 int longspec_hta_selftest_wait_timeout(void *workspace, cudaStream_t stream) {
@@ -545,6 +580,7 @@ int longspec_hta_get_status(void *workspace, cudaStream_t stream) {
     if (word & hta::kStatusBadParent) return LONGSPEC_HTA_ERR_BAD_PARENT;
     if (word & hta::kStatusPrefixLenRange) return LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE;
     if (word & hta::kStatusPipelineTimeout) return LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT;
+    if (word & hta::kStatusBadBlock) return LONGSPEC_HTA_ERR_BAD_BLOCK;
     if (word & hta::kStatusInternal) return LONGSPEC_HTA_ERR_INTERNAL;
     return LONGSPEC_HTA_OK;
 }

@@ -18,6 +18,7 @@ enum : uint32_t {
     kStatusPrefixLenRange = 1u << 1,
     kStatusPipelineTimeout = 1u << 2,
     kStatusInternal = 1u << 3,          // a kernel precondition did not hold
+    kStatusBadBlock = 1u << 4,          // a paged-cache block id out of range
 };
 
 constexpr int kStatusBytes = 256;   // status region at the start of a workspace

@@ -47,6 +47,11 @@ struct PrefixParams {
     const int32_t *prefix_len;
     float *o_part, *lse_part;         // [rows][S][D], [rows][S]
     uint32_t *status;
+    // Paged prefix K/V (tcgen05 kernel only): null block_table = contiguous
+    // [B][Hkv][L_cap][D]; else the caches are [num_blocks][Hkv][block_size][D]
+    // and the tensor maps' boxes are block_size rows high.
+    const int32_t *block_table;       // [B][max_blocks]
+    int block_size, max_blocks, num_blocks;
 };
 
 cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream);

@@ -197,7 +197,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 }  // namespace
 
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const PrefixParams p) {
@@ -270,6 +270,50 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         raise_status(p.status, kStatusPipelineTimeout);
     };
     const int kv_row0 = bk * p.L_cap + key_begin;
+    // Producer of a K or V ring from a paged cache, run by the whole warp.
+    // A 128-key tile is read with one block_size-row box per block and
+    // 64-column half, each landing at the block's rows of the swizzled stage
+    // (block_size * 128 bytes is a multiple of the 1024-byte swizzle period,
+    // so the layout is that of one tall box).  Per tile, lane 0 waits for the
+    // stage and posts the byte count; then lane i < 128/block_size issues the
+    // boxes of block i, whose id it read from the table one tile earlier.
+    // Blocks past L_b are read from the sequence's last block (their keys
+    // are masked); an id outside [0, num_blocks) is read as block 0 and
+    // flagged.  Returns the number of tiles issued.
+    auto paged_ring = [&](uint8_t *ring, const CUtensorMap *map, uint64_t *full, uint64_t *empty) {
+        const int bs = p.block_size, nb = kKeyTile / bs, kvh = bk % p.Hkv;
+        const int32_t *row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+        const int last = (L - 1) / bs;          // L >= 1: n_tiles > 0 here
+        auto fetch = [&](int key0) { return lane < nb ? row[min(key0 / bs + lane, last)] : 0; };
+        int id = fetch(key_begin);
+        int issued = 0;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j % C::NS;
+            int go = 0;                          // 1: proceed, 0: aborted, 2: wait ran out
+            if (lane == 0) {
+                go = *s_abort ? 0 : mbar_wait(empty + st, ((j / C::NS) & 1) ^ 1) ? 1 : 2;
+                if (go == 1) mbar_arrive_expect_tx(full + st, C::KV_BYTES);
+                if (go == 2) abort_cta();
+            }
+            go = __shfl_sync(0xffffffffu, go, 0);
+            if (go != 1) break;
+            if (lane < nb) {
+                int n = id;
+                if (n < 0 || n >= p.num_blocks) {
+                    raise_status(p.status, kStatusBadBlock);
+                    n = 0;
+                }
+                const int y = (n * p.Hkv + kvh) * bs;
+                uint8_t *stage = ring + st * C::KV_BYTES + lane * bs * 128;
+#pragma unroll
+                for (int h = 0; h < C::HALVES; ++h) tma_load_2d(stage + h * C::BOX_BYTES, map, full + st, h * 64, y);
+            }
+            id = fetch(key_begin + (j + 1) * C::BN);   // the next tile's block
+            issued = j + 1;
+        }
+        __syncwarp();
+        return issued;
+    };
     if (warp == kProducerKWarp) {
         // -------------------------------------------------------- TMA: Q, K
         regs_dec<kRegsOther>();
@@ -281,6 +325,15 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int h = 0; h < C::HALVES; ++h)
                 tma_load_2d(sq + h * C::BOX_BYTES, &tm_q, bars.q_full, h * 64, static_cast<int>(grow0));
+        }
+        if constexpr (PAGED) {
+            const int issued = paged_ring(smem + C::OFF_K, &tm_k, bars.k_full, bars.k_empty);
+            if (lane == 0 && *s_abort) {
+                mbar_wait(bars.q_full, 0);
+                for (int j = max(0, issued - C::NS); j < issued; ++j)
+                    mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1);
+            }
+        } else if (lane == 0) {
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % C::NS;
@@ -304,8 +357,14 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     } else if (warp == kProducerVWarp) {
         // ----------------------------------------------------------- TMA: V
         regs_dec<kRegsOther>();
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_v);
+        if (lane == 0) tma_prefetch_desc(&tm_v);
+        if constexpr (PAGED) {
+            const int issued = paged_ring(smem + C::OFF_V, &tm_v, bars.v_full, bars.v_empty);
+            if (lane == 0 && *s_abort) {
+                for (int j = max(0, issued - C::NS); j < issued; ++j)
+                    mbar_wait(bars.v_full + j % C::NS, (j / C::NS) & 1);
+            }
+        } else if (lane == 0) {
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % C::NS;
@@ -610,7 +669,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
-template <int D>
+template <int D, bool PAGED>
 cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                       const CUtensorMap &tm_v, cudaStream_t stream) {
     using C = TcCfg<D>;
@@ -621,7 +680,7 @@ cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUte
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(prefix_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(prefix_tc_kernel<D, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
@@ -638,13 +697,17 @@ cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefix_tc_kernel<D>, tm_q, tm_k, tm_v, p);
+    return cudaLaunchKernelEx(&cfg, prefix_tc_kernel<D, PAGED>, tm_q, tm_k, tm_v, p);
 }
 
 cudaError_t launch_prefix_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                              const CUtensorMap &tm_v, cudaStream_t stream) {
-    if (p.D == 128) return launch_tc<128>(p, tm_q, tm_k, tm_v, stream);
-    return launch_tc<64>(p, tm_q, tm_k, tm_v, stream);
+    const bool paged = p.block_table != nullptr;
+    if (p.D == 128)
+        return paged ? launch_tc<128, true>(p, tm_q, tm_k, tm_v, stream)
+                     : launch_tc<128, false>(p, tm_q, tm_k, tm_v, stream);
+    return paged ? launch_tc<64, true>(p, tm_q, tm_k, tm_v, stream)
+                 : launch_tc<64, false>(p, tm_q, tm_k, tm_v, stream);
 }
 
 }  // namespace hta

@@ -32,6 +32,7 @@ ERR_BAD_PARENT = -16
 ERR_PREFIX_LEN_RANGE = -17
 ERR_PIPELINE_TIMEOUT = -18
 ERR_INTERNAL = -19
+ERR_BAD_BLOCK = -20
 
 PREFIX_TCGEN05 = 0
 PREFIX_SIMT = 1
@@ -45,6 +46,7 @@ EXPORTED = [
     "longspec_hta_tree_mask", "longspec_hta_tree_partial", "longspec_hta_prefix_partial",
     "longspec_hta_get_status", "longspec_hta_verify_noalloc",
     "longspec_hta_selftest_wait_timeout", "longspec_hta_prefix_attention",
+    "longspec_hta_verify_paged", "longspec_hta_prefix_attention_paged",
 ]
 
 
@@ -64,6 +66,14 @@ class Dims(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("num_splits", ctypes.c_int), ("prefix_kernel", ctypes.c_int),
                 ("prefix_begin", ctypes.c_void_p), ("prefix_end", ctypes.c_void_p)]
+
+
+class PagedKV(ctypes.Structure):
+    """longspec_hta_paged_kv: caches [num_blocks][Hkv][block_size][D] bf16,
+    block_table [B][max_blocks] int32 (device pointers)."""
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("num_blocks", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("max_blocks", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -92,6 +102,9 @@ def load():
             lib.longspec_hta_verify.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
             lib.longspec_hta_verify_ex.argtypes = [pd] + [vp] * 9 + [vp, sz, ctypes.POINTER(Options), vp]
             lib.longspec_hta_prefix_attention.argtypes = [pd] + [vp] * 6 + [vp, sz, ctypes.POINTER(Options), vp]
+            pk = ctypes.POINTER(PagedKV)
+            lib.longspec_hta_verify_paged.argtypes = [pd, vp, pk] + [vp] * 6 + [vp, sz, ctypes.POINTER(Options), vp]
+            lib.longspec_hta_prefix_attention_paged.argtypes = [pd, vp, pk] + [vp] * 3 + [vp, sz, ctypes.POINTER(Options), vp]
             lib.longspec_hta_host_arena_bytes.argtypes = [pd]
             lib.longspec_hta_host_arena_bytes.restype = sz
             lib.longspec_hta_verify_host.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
@@ -218,6 +231,71 @@ def prefix_attention(q, k_prefix, v_prefix, prefix_len, *, out=None, lse=None, w
         ctypes.byref(dims), _ptr(q), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_len),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
         ctypes.byref(opts), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def _paged(k_cache, v_cache, block_table, dev):
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    if k_cache.dim() != 4 or k_cache.shape != v_cache.shape or block_table.dim() != 2:
+        raise ValueError("k/v_cache must be [num_blocks][Hkv][block_size][D], block_table [B][max_blocks]")
+    return PagedKV(_ptr(k_cache), _ptr(v_cache), _ptr(block_table), int(k_cache.shape[0]),
+                   int(k_cache.shape[2]), int(block_table.shape[1]))
+
+
+def _paged_dims(q, k_cache, L_cap, scale):
+    B, Hq, T, D = q.shape
+    return Dims(B, Hq, int(k_cache.shape[1]), D, T, int(L_cap), float(scale))
+
+
+def verify_paged(q, k_cache, v_cache, block_table, prefix_len, k_tree, v_tree, parent, *, L_cap,
+                 out=None, lse=None, workspace=None, scale: float = 0.0, num_splits: int = 0,
+                 prefix_events=None, stream=None):
+    """verify() with the prefix K/V in a paged cache: k/v_cache
+    [num_blocks][Hkv][block_size][D], block_table [B][max_blocks] (block ids
+    of each sequence in key order), L_cap the longest prefix allowed."""
+    dev = q.device
+    for t, n in ((q, "q"), (k_tree, "k_tree"), (v_tree, "v_tree")):
+        _need(t, n, torch.bfloat16, dev)
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    _need(parent, "parent", torch.int32, dev)
+    kv = _paged(k_cache, v_cache, block_table, dev)
+    dims = _paged_dims(q, k_cache, L_cap, scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev) if lse is None else lse
+    workspace = new_workspace(dims, num_splits, dev) if workspace is None else workspace
+    opts = Options(int(num_splits), PREFIX_TCGEN05,
+                   prefix_events[0].cuda_event if prefix_events else None,
+                   prefix_events[1].cuda_event if prefix_events else None)
+    rc = load().longspec_hta_verify_paged(
+        ctypes.byref(dims), _ptr(q), ctypes.byref(kv), _ptr(prefix_len), _ptr(k_tree), _ptr(v_tree),
+        _ptr(parent), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.byref(opts), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def prefix_attention_paged(q, k_cache, v_cache, block_table, prefix_len, *, L_cap, out=None,
+                           lse=None, workspace=None, scale: float = 0.0, num_splits: int = 0,
+                           prefix_events=None, stream=None):
+    """prefix_attention() with the prefix K/V in a paged cache."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    kv = _paged(k_cache, v_cache, block_table, dev)
+    dims = _paged_dims(q, k_cache, L_cap, scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev) if lse is None else lse
+    workspace = new_workspace(dims, num_splits, dev) if workspace is None else workspace
+    opts = Options(int(num_splits), PREFIX_TCGEN05,
+                   prefix_events[0].cuda_event if prefix_events else None,
+                   prefix_events[1].cuda_event if prefix_events else None)
+    rc = load().longspec_hta_prefix_attention_paged(
+        ctypes.byref(dims), _ptr(q), ctypes.byref(kv), _ptr(prefix_len), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), ctypes.byref(opts),
+        _stream(stream))
     _check(rc)
     return out, lse
 

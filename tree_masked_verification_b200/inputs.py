@@ -101,6 +101,9 @@ class Workload:
     # tokens attend to the prefix alone (longspec_hta_prefix_attention, the
     # draft model's cross-attention into the target's KV cache)
     kind: str = "verify"
+    # > 0: the prefix K/V in a paged cache of blocks of this many keys
+    # (longspec_hta_verify_paged / _prefix_attention_paged)
+    block_size: int = 0
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -241,9 +244,41 @@ WORKLOADS = {
     "ultra-256k-chain5": Workload("ultra-256k-chain5", B=1, Hq=32, Hkv=8,
                                   D=128, T=5, L_cap=262144, seed=5,
                                   tree="chain"),
+    # the Llama-3-8B call with the prefix in a paged cache of 16-key blocks
+    "llama3-8b-32k-paged16": Workload("llama3-8b-32k-paged16", B=1, Hq=32, Hkv=8, D=128,
+                                      T=68, L_cap=32768, seed=1, block_size=16),
     # the draft model's cross-attention into the Llama-3-8B target's KV
     # cache: 4 draft tokens per head, no tree keys
     "draft-xattn-32k": Workload("draft-xattn-32k", B=1, Hq=32, Hkv=8, D=128,
                                 T=4, L_cap=32768, seed=6, tree="chain",
                                 kind="prefix"),
 }
+
+
+def paged_cache(k_prefix: torch.Tensor, v_prefix: torch.Tensor, prefix_lens, block_size: int,
+                seed: int, spare_blocks: int = 3):
+    """The contiguous prefix K/V [B][Hkv][L_cap][D] laid out as a paged cache:
+    k/v_cache [num_blocks][Hkv][block_size][D] and block_table [B][max_blocks]
+    (int32), the blocks of all sequences shuffled by a seeded permutation,
+    with `spare_blocks` unused blocks of noise mixed in.  Table entries past
+    a sequence's last block are -1 (never read).  Pure data movement."""
+    B, Hkv, L_cap, D = k_prefix.shape
+    max_blocks = -(-L_cap // block_size)
+    lens = [int(x) for x in prefix_lens]
+    used = [-(-L // block_size) for L in lens]
+    n = sum(used) + spare_blocks
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(n, generator=g)
+    k_cache = torch.randn((n, Hkv, block_size, D), generator=g).to(torch.bfloat16)
+    v_cache = torch.randn((n, Hkv, block_size, D), generator=g).to(torch.bfloat16)
+    table = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        for i in range(used[b]):
+            blk = int(perm[nxt]); nxt += 1
+            table[b, i] = blk
+            k0, k1 = i * block_size, min((i + 1) * block_size, L_cap)
+            k_cache[blk, :, :k1 - k0] = k_prefix[b, :, k0:k1]
+            v_cache[blk, :, :k1 - k0] = v_prefix[b, :, k0:k1]
+    return k_cache, v_cache, table
+
