@@ -282,3 +282,27 @@ def paged_cache(k_prefix: torch.Tensor, v_prefix: torch.Tensor, prefix_lens, blo
             v_cache[blk, :, :k1 - k0] = v_prefix[b, :, k0:k1]
     return k_cache, v_cache, table
 
+
+
+def accept_inputs(B: int, T: int, V: int, seed: int, tree: str = "levels",
+                  widths: Tuple[int, ...] = LONGSPEC_TREE_SHAPE, p_match: float = 0.8):
+    """Seeded inputs of greedy tree acceptance: logits bf16 [B][T+1][V]
+    (row 0: the prefix end, row 1+i: after node i), draft_tokens and parent
+    int32 [B][T].  Every row gets a planted top token (logit 8 among N(0,1)
+    draws, so it is the row's unique maximum in practice); a node's draft
+    token is its parent row's planted token with probability p_match, else a
+    random token.  Also returns the planted tokens [B][T+1]."""
+    g = torch.Generator().manual_seed(seed)
+    logits = torch.randn((B, T + 1, V), generator=g)
+    top = torch.randint(0, V, (B, T + 1), generator=g)
+    logits.scatter_(2, top[..., None], 8.0)
+    wl = Workload("accept", B=B, Hq=1, Hkv=1, D=64, T=T, L_cap=0, seed=seed, tree=tree,
+                  widths=widths)
+    parent = torch.from_numpy(wl.parents().copy())
+    rows = torch.where(parent < 0, torch.zeros_like(parent), parent + 1).long()
+    want = torch.gather(top, 1, rows)
+    coin = torch.rand((B, T), generator=g) < p_match
+    other = torch.randint(0, V, (B, T), generator=g)
+    draft = torch.where(coin, want, other).to(torch.int32)
+    return dict(logits=logits.to(torch.bfloat16), draft_tokens=draft, parent=parent.to(torch.int32),
+                planted=top.to(torch.int32))
