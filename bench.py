@@ -32,7 +32,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from tree_masked_verification_b200 import hta  # noqa: E402
-from tree_masked_verification_b200.inputs import WORKLOADS, paged_cache  # noqa: E402
+from tree_masked_verification_b200.inputs import (ACCEPT_WORKLOADS, WORKLOADS, bf16_bits,  # noqa: E402
+                                                  accept_inputs, paged_cache)
 
 METRIC = "µs per layer verify-attention call; achieved HBM GB/s vs B200 peak @32k prefix"
 L2_BYTES = 126 * 1024 * 1024
@@ -446,6 +447,112 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------
+# greedy acceptance (the step after a verification call)
+# --------------------------------------------------------------------------
+def run_accept(args, world, rank, local):
+    """Latency of one greedy-acceptance call: argmax of B*(T+1) logits rows
+    of V bf16 values, then the tree walk.  HBM-bound on the logits read."""
+    B, T, V = ACCEPT_WORKLOADS[args.accept]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cpu = accept_inputs(B, T, V, seed=17 + rank, p_match=0.8)
+    lbytes = cpu["logits"].numel() * 2
+    n_sets = int(math.ceil(2 * L2_BYTES / lbytes)) + 1
+    base = {k: cpu[k].to(dev) for k in ("logits", "draft_tokens", "parent")}
+    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_sets - 1)]
+    ws = hta.new_accept_workspace(B, T, V, dev)
+    n_acc = torch.empty(B, dtype=torch.int32, device=dev)
+    path = torch.empty(B, T, dtype=torch.int32, device=dev)
+    bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(i):
+        s = sets[i % n_sets]
+        hta.accept_greedy(s["logits"], s["draft_tokens"], s["parent"], accept_len=n_acc, path=path,
+                          bonus=bonus, workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    if hta.get_status(ws) != hta.OK:
+        raise RuntimeError("device status error during warm-up")
+    sampler = ClockSampler(local if world > 1 else 0)
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t0.record(stream)
+    for i in range(args.steps):
+        call(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(world)
+    clocks = sampler.stop(wall0, wall1)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    if hta.get_status(ws) != hta.OK:
+        raise RuntimeError("device status error in the timed region")
+
+    # end to end: logits, tokens and parents from pinned host memory, the
+    # three results back to the host, every call
+    host = {k: cpu[k].pin_memory() for k in ("logits", "draft_tokens", "parent")}
+    n_e2e = min(args.e2e_steps * 10, args.steps)
+    outs = [torch.empty(B, dtype=torch.int32).pin_memory(), torch.empty(B, T, dtype=torch.int32).pin_memory(),
+            torch.empty(B, dtype=torch.int32).pin_memory()]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(n_e2e):
+        s = sets[i % n_sets]
+        for k in host:
+            s[k].copy_(host[k], non_blocking=True)
+        call(i)
+        for o, d in zip(outs, (n_acc, path, bonus)):
+            o.copy_(d, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    if rank != 0:
+        return
+    us = job_us_per_call(elapsed_ms, args.steps, world)
+    peak, peak_kind = peaks()
+    abytes = lbytes + 2 * B * T * 4 + 3 * B * 4 + B * T * 4
+    achieved = abytes / (elapsed_ms / args.steps * 1e-3) / 1e9
+    line = {
+        "metric": "greedy tree acceptance latency per call", "value": us, "unit": "µs",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) logits, one planted "
+        "maximum per row; LongSpec 4/16/16/16/16 tree; draft token = parent row's maximum w.p. 0.8)",
+        "config": {"workload": args.accept, "B": B, "T": T, "V": V, "input_sets": n_sets,
+                   "l2": f"{n_sets} rotating logits sets ({n_sets * lbytes / 1e6:.0f} MB > L2)"},
+        "roofline": {"bound": "hbm", "kernel": "argmax_slices_kernel + accept_kernel",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "algorithmic_bytes": abytes},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "e2e": {"value": job_us_per_call(e2e_ms, n_e2e, world), "unit": "µs",
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+                "d2h_bytes_per_step": sum(o.numel() * 4 for o in outs), "steps": n_e2e},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle.accept as oracle_accept
+        bits = bf16_bits(cpu["logits"])
+        tok, par = cpu["draft_tokens"].numpy(), cpu["parent"].numpy()
+        n, t_cpu = 0, time.perf_counter()
+        while n == 0 or time.perf_counter() - t_cpu < min(args.cpu_budget, 5.0):
+            oracle_accept.accept_greedy(bits, tok, par)
+            n += 1
+        line["cpu_baseline"] = {"value": (time.perf_counter() - t_cpu) / n * 1e6, "unit": "µs",
+                                "cores": 1, "kind": "oracle",
+                                "sample": f"{n} whole calls of the numpy oracle on the same inputs"}
+    print(json.dumps(line), flush=True)
+
+
 def run_e2e(args, w, cpu, dims, dev, stream, world):
     if w.block_size:
         names = ("q", "k_cache", "v_cache", "block_table", "prefix_len") + (
@@ -529,6 +636,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--accept", default=None, choices=sorted(ACCEPT_WORKLOADS),
+                    help="time greedy acceptance on this workload instead of attention")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -539,7 +648,10 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_ours(args, world, rank, local)
+        if args.accept:
+            run_accept(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -310,6 +310,34 @@ LONGSPEC_HTA_API int longspec_hta_prefix_attention_paged(const longspec_hta_dims
                                 void *out, float *lse, void *workspace, size_t workspace_bytes,
                                 const longspec_hta_options *opts, cudaStream_t stream);
 
+/* Greedy (temperature 0) acceptance of the speculated tree against the
+ * target model's logits: the step after verification attention.  LongSpec
+ * runs at temperature 0 (LongSpec README, "Inference": --temperature 0), so
+ * the target's token after a position is the argmax of its logits there.
+ * Node i of tree b is accepted when every node on its root path carries
+ * the target's argmax token at that node's parent position:
+ *   logits       bf16 [B][T+1][V], device: row 0 is the prefix end (judges
+ *                the root-level nodes, parent -1), row 1+i the position
+ *                after node i;
+ *   draft_tokens int32 [B][T], parent int32 [B][T] (as in verify);
+ *   accept_len   int32 [B]: depth of the deepest accepted node, 0 if none;
+ *   path         int32 [B][T]: its root path, node ids from depth 1, then -1;
+ *   bonus        int32 [B]: the target's argmax at the last accepted position
+ *                (row 0 when nothing is accepted), the token emitted after
+ *                the accepted ones.
+ * Among equally deep accepted nodes the smallest id wins; argmax ties go to
+ * the smallest token id; a NaN logit counts as -inf.  workspace: device, 16-byte
+ * aligned, longspec_hta_accept_workspace_bytes bytes (status word first).
+ * Errors: INVALID_DIMS (B, T, V < 1, B*(T+1) > 65535), T_TOO_LARGE,
+ * NULL_POINTER, MISALIGNED (logits and workspace 16 bytes, the int32 arrays
+ * 4 bytes), WORKSPACE_TOO_SMALL; a bad parent array gives accept_len 0 and
+ * LONGSPEC_HTA_ERR_BAD_PARENT from longspec_hta_get_status. */
+LONGSPEC_HTA_API size_t longspec_hta_accept_workspace_bytes(int B, int T, int V);
+LONGSPEC_HTA_API int longspec_hta_accept_greedy(int B, int T, int V, const void *logits,
+                                const int32_t *draft_tokens, const int32_t *parent,
+                                int32_t *accept_len, int32_t *path, int32_t *bonus,
+                                void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, reads and clears the status word of `workspace`,
  * and returns LONGSPEC_HTA_OK or the first device-detected error. */
 LONGSPEC_HTA_API int longspec_hta_get_status(void *workspace, cudaStream_t stream);

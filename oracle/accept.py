@@ -13,7 +13,8 @@ node's parent position.  The emitted tokens are the deepest accepted chain
 plus one token the target adds after it (its argmax at the chain's last
 position).  Readings where the pages are silent (stated in the design notes):
 the smallest node id wins among equally deep accepted nodes; argmax ties go
-to the smallest token id; a root-level node (parent -1) is judged at the
+to the smallest token id; a NaN logit counts as -inf (so a row of NaNs and
+-infs picks its first entry); a root-level node (parent -1) is judged at the
 prefix-end position.
 
 Plain numpy, one sequence at a time, in the order of the definition.
@@ -33,8 +34,11 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 def argmax_rows(logits_bits: np.ndarray) -> np.ndarray:
-    """First index of the largest value of every row (bf16 bits, [..., V])."""
-    return np.argmax(bf16_to_f64(logits_bits), axis=-1).astype(np.int64)
+    """First index of the largest value of every row (bf16 bits, [..., V]),
+    NaN read as -inf."""
+    x = bf16_to_f64(logits_bits)
+    x = np.where(np.isnan(x), -np.inf, x)
+    return np.argmax(x, axis=-1).astype(np.int64)
 
 
 def accept_greedy(logits_bits: np.ndarray, draft_tokens: np.ndarray, parent: np.ndarray):

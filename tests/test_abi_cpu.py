@@ -164,3 +164,34 @@ def test_paged_calls_reject_bad_arguments_on_host(lib):
     assert call(hta.PagedKV(**{**base, "num_blocks": 0})) == hta.ERR_INVALID_DIMS
     simt = hta.Options(0, hta.PREFIX_SIMT, None, None)
     assert call(hta.PagedKV(**base), simt) == hta.ERR_INVALID_OPTION
+
+
+def test_accept_rejects_bad_arguments_on_host(lib):
+    """Greedy acceptance: workspace size formula (status word + 32 slice
+    partials of 8 bytes per logits row), dims, NULL, alignment and
+    workspace checks, all taken before any device call."""
+    B, T, V = 4, 68, 128256
+    need = lib.longspec_hta_accept_workspace_bytes(B, T, V)
+    assert need == 256 + B * (T + 1) * 32 * 8
+    assert lib.longspec_hta_accept_workspace_bytes(0, T, V) == 0
+    assert lib.longspec_hta_accept_workspace_bytes(B, 257, V) == 0
+
+    def call(B=B, T=T, V=V, ptrs=None, ws_bytes=need):
+        p = ptrs or [4096 * (i + 1) for i in range(7)]   # logits, tok, parent, len, path, bonus, ws
+        return lib.longspec_hta_accept_greedy(B, T, V, *p, ws_bytes, None)
+
+    assert call(B=0) == hta.ERR_INVALID_DIMS
+    assert call(V=0) == hta.ERR_INVALID_DIMS
+    assert call(B=1000, T=100) == hta.ERR_INVALID_DIMS     # more than 65535 logits rows
+    assert call(T=257) == hta.ERR_T_TOO_LARGE
+    for k in range(7):
+        p = [4096 * (i + 1) for i in range(7)]
+        p[k] = None
+        assert call(ptrs=p) == hta.ERR_NULL_POINTER
+    p = [4096 * (i + 1) for i in range(7)]
+    p[0] += 8                                             # logits need 16 bytes
+    assert call(ptrs=p) == hta.ERR_MISALIGNED
+    p = [4096 * (i + 1) for i in range(7)]
+    p[3] += 2                                             # int32 arrays need 4 bytes
+    assert call(ptrs=p) == hta.ERR_MISALIGNED
+    assert call(ws_bytes=need - 1) == hta.ERR_WORKSPACE_TOO_SMALL

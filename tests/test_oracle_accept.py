@@ -122,3 +122,15 @@ def test_every_shape_of_a_small_tree():
                 if all(mask >> j & 1 for j in chain):
                     best = max(best, len(chain))
             assert length[0] == best
+
+
+def test_nan_counts_as_minus_inf():
+    """NaN logits: the first maximum of the row with every NaN read as -inf;
+    a row of NaNs and -infs picks its first entry (token 0)."""
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    vals = np.array([[[nan, 1.0, 3.0, nan], [nan, -inf, nan, -inf], [nan, nan, nan, nan]]],
+                    dtype=np.float32)
+    bits = (vals.view(np.uint32) >> 16).astype(np.uint16)
+    assert list(A.argmax_rows(bits)[0]) == [2, 0, 0]
+    length, path, bonus = A.accept_greedy(bits, np.array([[2, 0]]), np.array([[-1, 0]]))
+    assert length[0] == 2 and list(path[0]) == [0, 1] and bonus[0] == 0

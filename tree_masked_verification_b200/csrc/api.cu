@@ -560,6 +560,59 @@ int longspec_hta_prefix_attention_paged(const longspec_hta_dims *dims, const voi
                          workspace, workspace_bytes, opts, stream, true);
 }
 
+// ---- greedy acceptance ------------------------------------------------------
+namespace {
+constexpr int kAcceptMaxSlices = 32;
+// slices per logits row: enough CTAs to keep every SM streaming
+int accept_slices(int B, int T, int V, int num_sms) {
+    const long long rows = 1LL * B * (T + 1);
+    long long want = (4LL * num_sms + rows - 1) / rows;
+    want = std::min<long long>(want, (V + 2047) / 2048);     // at least 2048 elements a slice
+    return static_cast<int>(std::max<long long>(1, std::min<long long>(want, kAcceptMaxSlices)));
+}
+}  // namespace
+
+size_t longspec_hta_accept_workspace_bytes(int B, int T, int V) {
+    if (B < 1 || T < 1 || T > LONGSPEC_HTA_T_MAX || V < 1) return 0;
+    const size_t rows = static_cast<size_t>(B) * (T + 1);
+    return hta::kStatusBytes + rows * kAcceptMaxSlices * (sizeof(float) + sizeof(int));
+}
+
+int longspec_hta_accept_greedy(int B, int T, int V, const void *logits, const int32_t *draft_tokens,
+                               const int32_t *parent, int32_t *accept_len, int32_t *path, int32_t *bonus,
+                               void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (B < 1 || T < 1 || V < 1 || 1LL * B * (T + 1) > 65535 || 1LL * B * (T + 1) * V >= (1LL << 40))
+        return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    if (T > LONGSPEC_HTA_T_MAX) return LONGSPEC_HTA_ERR_T_TOO_LARGE;
+    const void *ptrs[] = {logits, draft_tokens, parent, accept_len, path, bonus, workspace};
+    for (const void *q : ptrs) {
+        if (!q) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if ((reinterpret_cast<uintptr_t>(q) & 3u) != 0) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    if (!aligned16(logits) || !aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    if (workspace_bytes < longspec_hta_accept_workspace_bytes(B, T, V)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo di;
+    int rc;
+    if ((rc = current_device(&di))) return rc;
+    hta::AcceptParams p{};
+    p.B = B; p.T = T; p.V = V;
+    p.n_slices = accept_slices(B, T, V, di.num_sms);
+    p.slice = ((V + p.n_slices - 1) / p.n_slices + 7) / 8 * 8;
+    p.n_slices = (V + p.slice - 1) / p.slice;
+    p.logits = static_cast<const __nv_bfloat16 *>(logits);
+    p.draft_tokens = draft_tokens;
+    p.parent = parent;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t rows = static_cast<size_t>(B) * (T + 1);
+    p.status = reinterpret_cast<uint32_t *>(ws);
+    p.part_v = reinterpret_cast<float *>(ws + hta::kStatusBytes);
+    p.part_i = reinterpret_cast<int *>(ws + hta::kStatusBytes + rows * kAcceptMaxSlices * sizeof(float));
+    p.accept_len = accept_len;
+    p.path = path;
+    p.bonus = bonus;
+    return hta::launch_accept(p, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
 int longspec_hta_selftest_wait_timeout(void *workspace, cudaStream_t stream) {
     if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
     if (!aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;

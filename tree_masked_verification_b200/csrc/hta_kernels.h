@@ -54,6 +54,19 @@ struct PrefixParams {
     int block_size, max_blocks, num_blocks;
 };
 
+// Greedy (temperature-0) acceptance of a speculated tree.  logits bf16
+// [B][T+1][V]: row 0 = the prefix end, row 1+i = the position after node i.
+struct AcceptParams {
+    int B, T, V;
+    int n_slices, slice;              // argmax slices per row, elements per slice (multiple of 8)
+    const __nv_bfloat16 *logits;
+    const int32_t *draft_tokens, *parent;   // [B][T]
+    float *part_v;                    // [B*(T+1)][n_slices] slice maxima
+    int *part_i;                      // [B*(T+1)][n_slices] their first indices
+    int32_t *accept_len, *path, *bonus;     // [B], [B][T], [B]
+    uint32_t *status;
+};
+cudaError_t launch_accept(const AcceptParams &p, cudaStream_t stream);
 cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream);
 // One bounded wait that is left to run out; sets kStatusPipelineTimeout.
 cudaError_t launch_wait_timeout_selftest(uint32_t *status, cudaStream_t stream);

@@ -287,6 +287,160 @@ tree_merge_kernel(TreeMergeParams p) {
     else tree_row<64>(p, s_anc, b, kvh, rr, bad);
 }
 
+// ------------------------------------------------------- greedy acceptance
+// Temperature-0 verification of the speculated tree against the target's
+// logits: node i is accepted when every node on its root path carries the
+// target's argmax token at that node's parent position; the deepest accepted
+// chain (smallest id among equally deep nodes) and the target's argmax after
+// it are the output.  Argmax ties go to the smallest token id; a NaN logit
+// never wins.
+
+namespace {
+
+struct ArgBest {
+    float v;
+    int i;
+};
+
+// (v, i) beats (bv, bi): larger value, or the same value at a smaller index;
+// a NaN counts as -inf (fmaxf returns the non-NaN operand)
+__device__ __forceinline__ void arg_take(ArgBest &b, float v, int i) {
+    v = fmaxf(v, -INFINITY);
+    if (v > b.v || (v == b.v && i < b.i)) { b.v = v; b.i = i; }
+}
+
+__device__ __forceinline__ void arg_take8(ArgBest &b, uint4 u, int i0) {
+    arg_take(b, bf16_lo(u.x), i0 + 0); arg_take(b, bf16_hi(u.x), i0 + 1);
+    arg_take(b, bf16_lo(u.y), i0 + 2); arg_take(b, bf16_hi(u.y), i0 + 3);
+    arg_take(b, bf16_lo(u.z), i0 + 4); arg_take(b, bf16_hi(u.z), i0 + 5);
+    arg_take(b, bf16_lo(u.w), i0 + 6); arg_take(b, bf16_hi(u.w), i0 + 7);
+}
+
+constexpr int kArgThreads = 256;
+
+}  // namespace
+
+// Slice `blockIdx.x` of row `blockIdx.y` of logits [rows][V] (bf16): its
+// (max, first index) into part[row][slice].  Slices are `slice` elements
+// long (a multiple of 8); rows whose start is 16-byte aligned are read with
+// 16-byte loads, four in flight per thread.
+__global__ void __launch_bounds__(kArgThreads)
+argmax_slices_kernel(const __nv_bfloat16 *logits, int V, int slice, float *part_v, int *part_i) {
+    // the logits may come from the previous kernel on the stream
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const size_t row = blockIdx.y;
+    const int s = blockIdx.x, n_slices = gridDim.x;
+    const int lo = s * slice, hi = min(V, lo + slice);
+    const __nv_bfloat16 *x = logits + row * static_cast<size_t>(V);
+    ArgBest b{-INFINITY, INT_MAX};
+    if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+        const int c_lo = lo / 8, c_hi = hi / 8;            // whole 8-element chunks
+        int c = c_lo + threadIdx.x;
+        for (; c + 3 * kArgThreads < c_hi; c += 4 * kArgThreads) {
+            const uint4 u0 = __ldcs(xv + c), u1 = __ldcs(xv + c + kArgThreads);
+            const uint4 u2 = __ldcs(xv + c + 2 * kArgThreads), u3 = __ldcs(xv + c + 3 * kArgThreads);
+            arg_take8(b, u0, 8 * c);
+            arg_take8(b, u1, 8 * (c + kArgThreads));
+            arg_take8(b, u2, 8 * (c + 2 * kArgThreads));
+            arg_take8(b, u3, 8 * (c + 3 * kArgThreads));
+        }
+        for (; c < c_hi; c += kArgThreads) arg_take8(b, __ldcs(xv + c), 8 * c);
+        for (int i = c_hi * 8 + threadIdx.x; i < hi; i += kArgThreads) arg_take(b, __bfloat162float(x[i]), i);
+    } else {
+        for (int i = lo + threadIdx.x; i < hi; i += kArgThreads) arg_take(b, __bfloat162float(x[i]), i);
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ArgBest t{__shfl_xor_sync(0xffffffffu, b.v, o), __shfl_xor_sync(0xffffffffu, b.i, o)};
+        arg_take(b, t.v, t.i);
+    }
+    __shared__ ArgBest s_best[kArgThreads / 32];
+    if (threadIdx.x % 32 == 0) s_best[threadIdx.x / 32] = b;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kArgThreads / 32; ++w) arg_take(b, s_best[w].v, s_best[w].i);
+        part_v[row * n_slices + s] = b.v;
+        part_i[row * n_slices + s] = b.i;
+    }
+}
+
+// One CTA (kTMax threads, thread i = node i) per sequence b.
+__global__ void __launch_bounds__(kThreads)
+accept_kernel(AcceptParams p) {
+    __shared__ int s_jump[kTMax];
+    __shared__ uint32_t s_anc[kTMax][kMaskWords];
+    __shared__ int s_flag;
+    __shared__ int s_amax[kTMax + 1];
+    __shared__ uint32_t s_match[kMaskWords];
+    __shared__ int s_best;
+    const int b = blockIdx.x, i = threadIdx.x, T = p.T, W = (T + 31) / 32;
+    // the mask needs only parent[]: built while the argmax grid runs
+    const bool bad = build_tree_mask(p.parent + static_cast<size_t>(b) * T, T, s_jump, s_anc, &s_flag);
+    if (i < kMaskWords) s_match[i] = 0u;
+    if (i == 0) s_best = -1;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // argmax of row r of this sequence from its slices
+    for (int r = i; r <= T; r += blockDim.x) {
+        const size_t row = static_cast<size_t>(b) * (T + 1) + r;
+        ArgBest best{-INFINITY, INT_MAX};
+        for (int s = 0; s < p.n_slices; ++s)
+            arg_take(best, p.part_v[row * p.n_slices + s], p.part_i[row * p.n_slices + s]);
+        s_amax[r] = best.i == INT_MAX ? 0 : best.i;
+    }
+    __syncthreads();
+    if (i < T && !bad) {
+        const int par = p.parent[static_cast<size_t>(b) * T + i];
+        if (p.draft_tokens[static_cast<size_t>(b) * T + i] == s_amax[par < 0 ? 0 : par + 1])
+            atomicOr(&s_match[i / 32], 1u << (i % 32));
+    }
+    __syncthreads();
+    int depth = 0;
+    if (i < T && !bad) {
+        bool accepted = true;
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w)
+            if (w < W) {
+                depth += __popc(s_anc[i][w]);
+                accepted = accepted && (s_anc[i][w] & ~s_match[w]) == 0u;
+            }
+        // deepest first, then the smallest id
+        if (accepted) atomicMax(&s_best, (depth << 16) | (0xFFFF - i));
+    }
+    __syncthreads();
+    const int best = s_best < 0 ? -1 : 0xFFFF - (s_best & 0xFFFF);
+    const int len = best < 0 ? 0 : s_best >> 16;
+    int32_t *path = p.path + static_cast<size_t>(b) * T;
+    if (i < T) {
+        if (i >= len) path[i] = -1;
+        if (best >= 0 && (s_anc[best][i / 32] >> (i % 32) & 1u)) path[depth - 1] = i;
+    }
+    if (i == 0) {
+        p.accept_len[b] = len;
+        p.bonus[b] = s_amax[best < 0 ? 0 : best + 1];
+        if (bad) raise_status(p.status, kStatusBadParent);
+    }
+}
+
+cudaError_t launch_accept(const AcceptParams &p, cudaStream_t stream) {
+    const int rows = p.B * (p.T + 1);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.stream = stream;
+    cfg.gridDim = dim3(p.n_slices, rows);
+    cfg.blockDim = dim3(kArgThreads);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, argmax_slices_kernel, p.logits, p.V, p.slice, p.part_v, p.part_i);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(p.B);
+    cfg.blockDim = dim3(kThreads);
+    return cudaLaunchKernelEx(&cfg, accept_kernel, p);
+}
+
 cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];

@@ -47,6 +47,7 @@ EXPORTED = [
     "longspec_hta_get_status", "longspec_hta_verify_noalloc",
     "longspec_hta_selftest_wait_timeout", "longspec_hta_prefix_attention",
     "longspec_hta_verify_paged", "longspec_hta_prefix_attention_paged",
+    "longspec_hta_accept_workspace_bytes", "longspec_hta_accept_greedy",
 ]
 
 
@@ -115,6 +116,9 @@ def load():
             lib.longspec_hta_get_status.argtypes = [vp, vp]
             lib.longspec_hta_selftest_wait_timeout.argtypes = [vp, vp]
             lib.longspec_hta_chunking.argtypes = [pd, ci, ctypes.POINTER(ci), ctypes.POINTER(ci)]
+            lib.longspec_hta_accept_workspace_bytes.argtypes = [ci, ci, ci]
+            lib.longspec_hta_accept_workspace_bytes.restype = sz
+            lib.longspec_hta_accept_greedy.argtypes = [ci, ci, ci] + [vp] * 6 + [vp, sz, vp]
             _lib = lib
     return _lib
 
@@ -374,6 +378,46 @@ def prefix_partial(q, k_prefix, v_prefix, prefix_len, *, scale: float = 0.0,
     if S_out.value != S:
         raise RuntimeError(f"split count mismatch: library {S_out.value}, binding {S}")
     return o, l, chunk_keys
+
+
+def accept_workspace_bytes(B: int, T: int, V: int) -> int:
+    return int(load().longspec_hta_accept_workspace_bytes(int(B), int(T), int(V)))
+
+
+def new_accept_workspace(B: int, T: int, V: int, device=None) -> torch.Tensor:
+    n = accept_workspace_bytes(B, T, V)
+    if n == 0:
+        raise HtaError(ERR_INVALID_DIMS)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def accept_greedy(logits, draft_tokens, parent, *, accept_len=None, path=None, bonus=None,
+                  workspace=None, stream=None):
+    """Greedy (temperature 0) acceptance of the draft tree.
+
+    logits bf16 [B][T+1][V] (row 0: the prefix end, row 1+i: after node i),
+    draft_tokens and parent int32 [B][T].  Returns (accept_len int32 [B],
+    path int32 [B][T] padded with -1, bonus int32 [B])."""
+    _need(logits, "logits", torch.bfloat16)
+    dev = logits.device
+    _need(draft_tokens, "draft_tokens", torch.int32, dev)
+    _need(parent, "parent", torch.int32, dev)
+    B, T1, V = logits.shape
+    T = T1 - 1
+    if tuple(draft_tokens.shape) != (B, T) or tuple(parent.shape) != (B, T):
+        raise ValueError(f"draft_tokens/parent must be [{B}][{T}]")
+    if accept_len is None:
+        accept_len = torch.empty(B, dtype=torch.int32, device=dev)
+    if path is None:
+        path = torch.empty(B, T, dtype=torch.int32, device=dev)
+    if bonus is None:
+        bonus = torch.empty(B, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_accept_workspace(B, T, V, dev)
+    _check(load().longspec_hta_accept_greedy(
+        B, T, V, _ptr(logits), _ptr(draft_tokens), _ptr(parent), _ptr(accept_len), _ptr(path),
+        _ptr(bonus), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return accept_len, path, bonus
 
 
 def selftest_wait_timeout(workspace: torch.Tensor, stream=None) -> int:

@@ -284,6 +284,14 @@ def paged_cache(k_prefix: torch.Tensor, v_prefix: torch.Tensor, prefix_lens, blo
 
 
 
+# greedy acceptance after a verification call: (B, T, V); T is the LongSpec
+# tree's 68 nodes, V the target model's vocabulary
+ACCEPT_WORKLOADS = {
+    "accept-llama3-t68": (1, 68, 128256),
+    "accept-vicuna-b8": (8, 68, 32000),
+}
+
+
 def accept_inputs(B: int, T: int, V: int, seed: int, tree: str = "levels",
                   widths: Tuple[int, ...] = LONGSPEC_TREE_SHAPE, p_match: float = 0.8):
     """Seeded inputs of greedy tree acceptance: logits bf16 [B][T+1][V]
