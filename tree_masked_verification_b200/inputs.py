@@ -256,16 +256,18 @@ WORKLOADS = {
 
 
 def paged_cache(k_prefix: torch.Tensor, v_prefix: torch.Tensor, prefix_lens, block_size: int,
-                seed: int, spare_blocks: int = 3):
+                seed: int, spare_blocks: int = 3, reserve: int = 0):
     """The contiguous prefix K/V [B][Hkv][L_cap][D] laid out as a paged cache:
     k/v_cache [num_blocks][Hkv][block_size][D] and block_table [B][max_blocks]
     (int32), the blocks of all sequences shuffled by a seeded permutation,
-    with `spare_blocks` unused blocks of noise mixed in.  Table entries past
-    a sequence's last block are -1 (never read).  Pure data movement."""
+    with `spare_blocks` unused blocks of noise mixed in.  Each sequence gets
+    blocks for its L_b keys plus `reserve` more positions (room for tokens
+    appended later), capped at L_cap.  Table entries past a sequence's last
+    block are -1 (never read).  Pure data movement."""
     B, Hkv, L_cap, D = k_prefix.shape
     max_blocks = -(-L_cap // block_size)
     lens = [int(x) for x in prefix_lens]
-    used = [-(-L // block_size) for L in lens]
+    used = [-(-min(L + reserve, L_cap) // block_size) for L in lens]
     n = sum(used) + spare_blocks
     g = torch.Generator().manual_seed(seed)
     perm = torch.randperm(n, generator=g)
@@ -314,3 +316,32 @@ def accept_inputs(B: int, T: int, V: int, seed: int, tree: str = "levels",
     draft = torch.where(coin, want, other).to(torch.int32)
     return dict(logits=logits.to(torch.bfloat16), draft_tokens=draft, parent=parent.to(torch.int32),
                 planted=top.to(torch.int32))
+
+
+def commit_inputs(w: "Workload", seed: int, full_prefix: bool = False):
+    """Seeded inputs of the KV commit after acceptance: the workload's
+    prefix cache, prefix lengths and tree K/V (``w.generate()``), plus, per
+    sequence, an accepted path: the root path of a node drawn uniformly from
+    the tree (node ids from depth 1), or no path with probability 1/8.
+    Returns the generate() dict plus accept_len int32 [B] and path int32
+    [B][T] (-1 past accept_len)."""
+    inp = w.generate()
+    g = torch.Generator().manual_seed(seed)
+    par = inp["parent"].numpy()
+    B, T = par.shape
+    path = np.full((B, T), -1, dtype=np.int32)
+    n = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        if torch.rand((), generator=g).item() < 0.125:
+            continue
+        j = int(torch.randint(0, T, (), generator=g))
+        chain = []
+        while j != -1:
+            chain.append(j)
+            j = int(par[b, j])
+        chain.reverse()
+        n[b] = len(chain)
+        path[b, :len(chain)] = chain
+    inp["accept_len"] = torch.from_numpy(n)
+    inp["path"] = torch.from_numpy(path)
+    return inp
