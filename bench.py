@@ -495,6 +495,40 @@ def run_accept(args, world, rank, local):
     if hta.get_status(ws) != hta.OK:
         raise RuntimeError("device status error in the timed region")
 
+    # acceptance followed by the KV commit of the accepted path (8 KV heads,
+    # D 128, contiguous cache) on the device, back to back: every call
+    # appends up to (tree depth) rows, so the cache is sized for all calls
+    Hkv, D = 8, 128
+    n_pipe = min(args.steps, 2000)
+    par = cpu["parent"].numpy()
+    depth = np.zeros(par.shape, dtype=np.int64)
+    for i in range(T):
+        depth[:, i] = np.where(par[:, i] < 0, 1, depth[np.arange(B), np.maximum(par[:, i], 0)] + 1)
+    L_cap = int((n_pipe + args.warmup + 1) * depth.max())
+    kcache = torch.zeros(B, Hkv, L_cap, D, dtype=torch.bfloat16, device=dev)
+    vcache = torch.zeros_like(kcache)
+    ktree = torch.randn(B, Hkv, T, D, device=dev).to(torch.bfloat16)
+    vtree = torch.randn_like(ktree)
+    lens = torch.zeros(B, dtype=torch.int32, device=dev)
+
+    def pipe(i):
+        call(i)
+        hta.commit(kcache, vcache, lens, ktree, vtree, n_acc, path, workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        pipe(i)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    p0.record(stream)
+    for i in range(n_pipe):
+        pipe(i)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    pipe_ms = max_over_ranks(p0.elapsed_time(p1), world)
+    if hta.get_status(ws) != hta.OK:
+        raise RuntimeError("device status error in the accept + commit region")
+
     # end to end: logits, tokens and parents from pinned host memory, the
     # three results back to the host, every call
     host = {k: cpu[k].pin_memory() for k in ("logits", "draft_tokens", "parent")}
@@ -535,6 +569,11 @@ def run_accept(args, world, rank, local):
                      "frac": achieved / peak, "traffic": None, "algorithmic_bytes": abytes},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
+        "accept_then_commit": {
+            "us_per_call": job_us_per_call(pipe_ms, n_pipe, world), "calls": n_pipe,
+            "gpu_launches": 3 * n_pipe,
+            "note": "accept_greedy + commit (8 KV heads, D 128, contiguous cache) per call, "
+                    "back to back; the prefix grows by the accepted length every call"},
         "e2e": {"value": job_us_per_call(e2e_ms, n_e2e, world), "unit": "µs",
                 "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
                 "d2h_bytes_per_step": sum(o.numel() * 4 for o in outs), "steps": n_e2e},

@@ -86,7 +86,8 @@ typedef enum {
     LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE = -17,   /* some prefix_len[b] outside [0, L_cap] */
     LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT = -18,   /* a bounded in-kernel wait ran out */
     LONGSPEC_HTA_ERR_INTERNAL = -19,           /* a kernel precondition failed (a library bug) */
-    LONGSPEC_HTA_ERR_BAD_BLOCK = -20           /* a block_table entry outside [0, num_blocks) */
+    LONGSPEC_HTA_ERR_BAD_BLOCK = -20,          /* a block_table entry outside [0, num_blocks) */
+    LONGSPEC_HTA_ERR_BAD_PATH = -21            /* accept_len outside [0, T] or a path entry outside [0, T) */
 } longspec_hta_status;
 
 /* Problem sizes of one call.  scale 0 means 1/sqrt(D); otherwise > 0. */
@@ -337,6 +338,42 @@ LONGSPEC_HTA_API int longspec_hta_accept_greedy(int B, int T, int V, const void 
                                 const int32_t *draft_tokens, const int32_t *parent,
                                 int32_t *accept_len, int32_t *path, int32_t *bonus,
                                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Commit of the accepted path: after verification and acceptance, the
+ * accepted tokens join the target's context, so their K/V rows (the tree
+ * keys the verification pass used) are appended to the KV cache right after
+ * the prefix and the prefix grows by the accepted length (LongSpec README,
+ * "Introduction": the target model verifies the speculated tree and keeps
+ * the accepted tokens; rejected branches are dropped).  For every sequence b
+ * with L_b = prefix_len[b], n_b = accept_len[b] and every KV head h:
+ *   cache_K[b][h][L_b + d] = k_tree[b][h][path[b][d]],  d < n_b (V alike),
+ * then prefix_len[b] = L_b + n_b (in place, on the device).  Cache rows past
+ * L_b + n_b are not touched.
+ *   dims: B, Hkv, D, T, L_cap as in verify (Hq and scale only validated);
+ *   k_prefix/v_prefix: the contiguous cache bf16 [B][Hkv][L_cap][D];
+ *   kv: a paged cache (position p of sequence b is row p % block_size of
+ *       block block_table[b][p / block_size]); the commit writes through
+ *       kv->k_cache and kv->v_cache, and the table must already map every
+ *       position below L_b + n_b;
+ *   prefix_len int32 [B] (read, then advanced); k_tree/v_tree bf16
+ *   [B][Hkv][T][D]; accept_len int32 [B] and path int32 [B][T] as written by
+ *   longspec_hta_accept_greedy (device; may come from the previous kernel on
+ *   the stream, no host synchronisation is needed);
+ *   workspace: device, at least 256 bytes (the status word).
+ * Host errors: NULL_POINTER, MISALIGNED (caches, tree K/V and workspace 16
+ * bytes; the int32 arrays 4 bytes), INVALID_DIMS, UNSUPPORTED_D,
+ * T_TOO_LARGE, WORKSPACE_TOO_SMALL.  Device errors leave the sequence
+ * unchanged (no row written, prefix_len kept) and set the status word:
+ * BAD_PATH (n_b outside [0, T] or a path entry outside [0, T)),
+ * PREFIX_LEN_RANGE (L_b outside [0, L_cap] or L_b + n_b > L_cap), BAD_BLOCK. */
+LONGSPEC_HTA_API int longspec_hta_commit(const longspec_hta_dims *dims, void *k_prefix, void *v_prefix,
+                                int32_t *prefix_len, const void *k_tree, const void *v_tree,
+                                const int32_t *accept_len, const int32_t *path, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+LONGSPEC_HTA_API int longspec_hta_commit_paged(const longspec_hta_dims *dims, const longspec_hta_paged_kv *kv,
+                                int32_t *prefix_len, const void *k_tree, const void *v_tree,
+                                const int32_t *accept_len, const int32_t *path, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
 
 /* Synchronises `stream`, reads and clears the status word of `workspace`,
  * and returns LONGSPEC_HTA_OK or the first device-detected error. */

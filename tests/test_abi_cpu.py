@@ -195,3 +195,41 @@ def test_accept_rejects_bad_arguments_on_host(lib):
     p[3] += 2                                             # int32 arrays need 4 bytes
     assert call(ptrs=p) == hta.ERR_MISALIGNED
     assert call(ws_bytes=need - 1) == hta.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_commit_rejects_bad_arguments_on_host(lib):
+    """KV commit: dims, NULL, alignment, paged descriptor and workspace
+    checks, all taken before any device call."""
+    d = _dims(L_cap=1024)
+    good = [4096 * (i + 1) for i in range(7)]   # k_prefix, v_prefix, prefix_len, k_tree, v_tree, len, path
+
+    def call(p=None, ws=4096 * 20, ws_bytes=256, dims=d):
+        p = good if p is None else p
+        return lib.longspec_hta_commit(ctypes.byref(dims), *p, ws, ws_bytes, None)
+
+    for k in range(7):
+        p = list(good)
+        p[k] = None
+        assert call(p) == hta.ERR_NULL_POINTER
+    p = list(good)
+    p[0] += 8                                   # the cache needs 16 bytes
+    assert call(p) == hta.ERR_MISALIGNED
+    p = list(good)
+    p[2] += 2                                   # int32 arrays need 4 bytes
+    assert call(p) == hta.ERR_MISALIGNED
+    assert call(ws=None) == hta.ERR_NULL_POINTER
+    assert call(ws_bytes=255) == hta.ERR_WORKSPACE_TOO_SMALL
+    assert call(dims=_dims(D=96)) == hta.ERR_UNSUPPORTED_D
+    assert call(dims=_dims(T=300)) == hta.ERR_T_TOO_LARGE
+
+    base = dict(k_cache=4096 * 30, v_cache=4096 * 31, block_table=4096 * 32, num_blocks=64,
+                block_size=16, max_blocks=64)
+
+    def paged(kv):
+        return lib.longspec_hta_commit_paged(ctypes.byref(d), None if kv is None else ctypes.byref(kv),
+                                             *good[2:], 4096 * 20, 256, None)
+
+    assert paged(None) == hta.ERR_NULL_POINTER
+    assert paged(hta.PagedKV(**{**base, "block_table": 0})) == hta.ERR_NULL_POINTER
+    assert paged(hta.PagedKV(**{**base, "block_size": 24})) == hta.ERR_INVALID_DIMS
+    assert paged(hta.PagedKV(**{**base, "max_blocks": 63})) == hta.ERR_INVALID_DIMS

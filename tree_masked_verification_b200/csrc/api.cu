@@ -270,6 +270,7 @@ const char *longspec_hta_strerror(int code) {
     case LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT: return "in-kernel wait timed out";
     case LONGSPEC_HTA_ERR_INTERNAL: return "internal kernel precondition failed";
     case LONGSPEC_HTA_ERR_BAD_BLOCK: return "a block_table entry is outside [0, num_blocks)";
+    case LONGSPEC_HTA_ERR_BAD_PATH: return "an accepted length or path entry is out of range";
     default: return "unknown status";
     }
 }
@@ -613,6 +614,75 @@ int longspec_hta_accept_greedy(int B, int T, int V, const void *logits, const in
     return hta::launch_accept(p, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
 }
 
+// ---- KV commit of the accepted path ----------------------------------------
+namespace {
+int run_commit(const longspec_hta_dims *dims, void *k_cache, void *v_cache,
+               const longspec_hta_paged_kv *kv, int32_t *prefix_len, const void *k_tree,
+               const void *v_tree, const int32_t *accept_len, const int32_t *path, void *workspace,
+               size_t workspace_bytes, cudaStream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (kv) {   // the commit writes the cache the descriptor points to
+        k_cache = const_cast<void *>(kv->k_cache);
+        v_cache = const_cast<void *>(kv->v_cache);
+    }
+    const void *big[] = {k_cache, v_cache, k_tree, v_tree, workspace};
+    for (const void *q : big) {
+        if (!q) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(q)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    const void *ints[] = {prefix_len, accept_len, path, kv ? static_cast<const void *>(kv->block_table) : path};
+    for (const void *q : ints) {
+        if (!q) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if ((reinterpret_cast<uintptr_t>(q) & 3u) != 0) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    if (kv) {
+        const int bs = kv->block_size;
+        if ((bs != 16 && bs != 32 && bs != 64 && bs != 128) || kv->num_blocks < 1 || kv->max_blocks < 1 ||
+            1LL * kv->max_blocks * bs < dims->L_cap ||
+            1LL * kv->num_blocks * dims->Hkv * bs + 128 >= (1LL << 31))
+            return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    }
+    if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    hta::CommitParams p{};
+    p.B = dims->B; p.Hkv = dims->Hkv; p.D = dims->D; p.T = dims->T; p.L_cap = dims->L_cap;
+    p.k_cache = static_cast<__nv_bfloat16 *>(k_cache);
+    p.v_cache = static_cast<__nv_bfloat16 *>(v_cache);
+    if (kv) {
+        p.block_table = kv->block_table;
+        p.block_size = kv->block_size;
+        p.max_blocks = kv->max_blocks;
+        p.num_blocks = kv->num_blocks;
+    }
+    p.prefix_len = prefix_len;
+    p.k_tree = static_cast<const __nv_bfloat16 *>(k_tree);
+    p.v_tree = static_cast<const __nv_bfloat16 *>(v_tree);
+    p.accept_len = accept_len;
+    p.path = path;
+    p.status = static_cast<uint32_t *>(workspace);
+    return hta::launch_commit(p, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+}  // namespace
+
+int longspec_hta_commit(const longspec_hta_dims *dims, void *k_prefix, void *v_prefix,
+                        int32_t *prefix_len, const void *k_tree, const void *v_tree,
+                        const int32_t *accept_len, const int32_t *path, void *workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+    return run_commit(dims, k_prefix, v_prefix, nullptr, prefix_len, k_tree, v_tree, accept_len, path,
+                      workspace, workspace_bytes, stream);
+}
+
+int longspec_hta_commit_paged(const longspec_hta_dims *dims, const longspec_hta_paged_kv *kv,
+                              int32_t *prefix_len, const void *k_tree, const void *v_tree,
+                              const int32_t *accept_len, const int32_t *path, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+    if (!kv) return LONGSPEC_HTA_ERR_NULL_POINTER;
+    return run_commit(dims, nullptr, nullptr, kv, prefix_len, k_tree, v_tree, accept_len, path,
+                      workspace, workspace_bytes, stream);
+}
+
 int longspec_hta_selftest_wait_timeout(void *workspace, cudaStream_t stream) {
     if (!workspace) return LONGSPEC_HTA_ERR_NULL_POINTER;
     if (!aligned16(workspace)) return LONGSPEC_HTA_ERR_MISALIGNED;
@@ -634,6 +704,7 @@ int longspec_hta_get_status(void *workspace, cudaStream_t stream) {
     if (word & hta::kStatusPrefixLenRange) return LONGSPEC_HTA_ERR_PREFIX_LEN_RANGE;
     if (word & hta::kStatusPipelineTimeout) return LONGSPEC_HTA_ERR_PIPELINE_TIMEOUT;
     if (word & hta::kStatusBadBlock) return LONGSPEC_HTA_ERR_BAD_BLOCK;
+    if (word & hta::kStatusBadPath) return LONGSPEC_HTA_ERR_BAD_PATH;
     if (word & hta::kStatusInternal) return LONGSPEC_HTA_ERR_INTERNAL;
     return LONGSPEC_HTA_OK;
 }

@@ -19,6 +19,7 @@ enum : uint32_t {
     kStatusPipelineTimeout = 1u << 2,
     kStatusInternal = 1u << 3,          // a kernel precondition did not hold
     kStatusBadBlock = 1u << 4,          // a paged-cache block id out of range
+    kStatusBadPath = 1u << 5,           // an accepted length or path entry out of range
 };
 
 constexpr int kStatusBytes = 256;   // status region at the start of a workspace

@@ -67,6 +67,19 @@ struct AcceptParams {
     uint32_t *status;
 };
 cudaError_t launch_accept(const AcceptParams &p, cudaStream_t stream);
+
+// Append the accepted path's tree K/V to the cache; prefix_len advances in place.
+struct CommitParams {
+    int B, Hkv, D, T, L_cap;
+    __nv_bfloat16 *k_cache, *v_cache;          // [B][Hkv][L_cap][D], or paged [num_blocks][Hkv][block_size][D]
+    const int32_t *block_table;                // [B][max_blocks], nullptr for a contiguous cache
+    int block_size, max_blocks, num_blocks;
+    int32_t *prefix_len;                       // [B], read and advanced
+    const __nv_bfloat16 *k_tree, *v_tree;      // [B][Hkv][T][D]
+    const int32_t *accept_len, *path;          // [B], [B][T]
+    uint32_t *status;
+};
+cudaError_t launch_commit(const CommitParams &p, cudaStream_t stream);
 cudaError_t launch_tree_merge(const TreeMergeParams &p, cudaStream_t stream);
 // One bounded wait that is left to run out; sets kStatusPipelineTimeout.
 cudaError_t launch_wait_timeout_selftest(uint32_t *status, cudaStream_t stream);

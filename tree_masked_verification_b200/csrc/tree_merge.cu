@@ -323,7 +323,7 @@ constexpr int kArgThreads = 256;
 // Slice `blockIdx.x` of row `blockIdx.y` of logits [rows][V] (bf16): its
 // (max, first index) into part[row][slice].  Slices are `slice` elements
 // long (a multiple of 8); rows whose start is 16-byte aligned are read with
-// 16-byte loads, four in flight per thread.
+// 16-byte loads, up to eight in flight per thread.
 __global__ void __launch_bounds__(kArgThreads)
 argmax_slices_kernel(const __nv_bfloat16 *logits, int V, int slice, float *part_v, int *part_i) {
     // the logits may come from the previous kernel on the stream
@@ -336,16 +336,16 @@ argmax_slices_kernel(const __nv_bfloat16 *logits, int V, int slice, float *part_
     if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
         const uint4 *xv = reinterpret_cast<const uint4 *>(x);
         const int c_lo = lo / 8, c_hi = hi / 8;            // whole 8-element chunks
-        int c = c_lo + threadIdx.x;
-        for (; c + 3 * kArgThreads < c_hi; c += 4 * kArgThreads) {
-            const uint4 u0 = __ldcs(xv + c), u1 = __ldcs(xv + c + kArgThreads);
-            const uint4 u2 = __ldcs(xv + c + 2 * kArgThreads), u3 = __ldcs(xv + c + 3 * kArgThreads);
-            arg_take8(b, u0, 8 * c);
-            arg_take8(b, u1, 8 * (c + kArgThreads));
-            arg_take8(b, u2, 8 * (c + 2 * kArgThreads));
-            arg_take8(b, u3, 8 * (c + 3 * kArgThreads));
+        // up to eight 16-byte loads in flight per thread, then their compares
+        for (int c = c_lo + threadIdx.x; c < c_hi; c += 8 * kArgThreads) {
+            uint4 u[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                u[k] = c + k * kArgThreads < c_hi ? __ldcs(xv + c + k * kArgThreads) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (c + k * kArgThreads < c_hi) arg_take8(b, u[k], 8 * (c + k * kArgThreads));
         }
-        for (; c < c_hi; c += kArgThreads) arg_take8(b, __ldcs(xv + c), 8 * c);
         for (int i = c_hi * 8 + threadIdx.x; i < hi; i += kArgThreads) arg_take(b, __bfloat162float(x[i]), i);
     } else {
         for (int i = lo + threadIdx.x; i < hi; i += kArgThreads) arg_take(b, __bfloat162float(x[i]), i);
@@ -381,13 +381,34 @@ accept_kernel(AcceptParams p) {
     if (i < kMaskWords) s_match[i] = 0u;
     if (i == 0) s_best = -1;
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // argmax of row r of this sequence from its slices
-    for (int r = i; r <= T; r += blockDim.x) {
-        const size_t row = static_cast<size_t>(b) * (T + 1) + r;
-        ArgBest best{-INFINITY, INT_MAX};
-        for (int s = 0; s < p.n_slices; ++s)
-            arg_take(best, p.part_v[row * p.n_slices + s], p.part_i[row * p.n_slices + s]);
-        s_amax[r] = best.i == INT_MAX ? 0 : best.i;
+    // argmax of row r of this sequence from its slices: warp w takes rows
+    // w, w + 8, ..., four rows at a time, lane s reads slice s (n_slices <= 32),
+    // so the partials of four rows are in flight at once
+    {
+        const int lane = i % 32, warp = i / 32;
+        const size_t row0 = static_cast<size_t>(b) * (T + 1);
+        for (int r0 = warp; r0 <= T; r0 += 4 * kWarps) {
+            ArgBest c[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = r0 + u * kWarps;
+                const bool live = r <= T && lane < p.n_slices;
+                const size_t k = (row0 + r) * p.n_slices + lane;
+                c[u].v = live ? p.part_v[k] : -INFINITY;
+                c[u].i = live ? p.part_i[k] : INT_MAX;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float v = __shfl_xor_sync(0xffffffffu, c[u].v, o);
+                    const int ix = __shfl_xor_sync(0xffffffffu, c[u].i, o);
+                    arg_take(c[u], v, ix);
+                }
+                const int r = r0 + u * kWarps;
+                if (lane == 0 && r <= T) s_amax[r] = c[u].i == INT_MAX ? 0 : c[u].i;
+            }
+        }
     }
     __syncthreads();
     if (i < T && !bad) {

@@ -33,6 +33,7 @@ ERR_PREFIX_LEN_RANGE = -17
 ERR_PIPELINE_TIMEOUT = -18
 ERR_INTERNAL = -19
 ERR_BAD_BLOCK = -20
+ERR_BAD_PATH = -21
 
 PREFIX_TCGEN05 = 0
 PREFIX_SIMT = 1
@@ -48,6 +49,7 @@ EXPORTED = [
     "longspec_hta_selftest_wait_timeout", "longspec_hta_prefix_attention",
     "longspec_hta_verify_paged", "longspec_hta_prefix_attention_paged",
     "longspec_hta_accept_workspace_bytes", "longspec_hta_accept_greedy",
+    "longspec_hta_commit", "longspec_hta_commit_paged",
 ]
 
 
@@ -119,6 +121,8 @@ def load():
             lib.longspec_hta_accept_workspace_bytes.argtypes = [ci, ci, ci]
             lib.longspec_hta_accept_workspace_bytes.restype = sz
             lib.longspec_hta_accept_greedy.argtypes = [ci, ci, ci] + [vp] * 6 + [vp, sz, vp]
+            lib.longspec_hta_commit.argtypes = [pd] + [vp] * 7 + [vp, sz, vp]
+            lib.longspec_hta_commit_paged.argtypes = [pd, pk] + [vp] * 5 + [vp, sz, vp]
             _lib = lib
     return _lib
 
@@ -418,6 +422,45 @@ def accept_greedy(logits, draft_tokens, parent, *, accept_len=None, path=None, b
         B, T, V, _ptr(logits), _ptr(draft_tokens), _ptr(parent), _ptr(accept_len), _ptr(path),
         _ptr(bonus), _ptr(workspace), workspace.numel(), _stream(stream)))
     return accept_len, path, bonus
+
+
+def _commit_dims(k_tree, L_cap):
+    B, Hkv, T, D = k_tree.shape
+    return Dims(B, Hkv, Hkv, D, T, int(L_cap), 0.0)
+
+
+def commit(k_prefix, v_prefix, prefix_len, k_tree, v_tree, accept_len, path, *, workspace=None,
+           stream=None):
+    """Append the accepted path's tree K/V rows to the contiguous cache
+    [B][Hkv][L_cap][D] after each prefix and advance prefix_len in place."""
+    for t, n in ((k_prefix, "k_prefix"), (v_prefix, "v_prefix"), (k_tree, "k_tree"), (v_tree, "v_tree")):
+        _need(t, n, torch.bfloat16, k_tree.device)
+    for t, n in ((prefix_len, "prefix_len"), (accept_len, "accept_len"), (path, "path")):
+        _need(t, n, torch.int32, k_tree.device)
+    dims = _commit_dims(k_tree, k_prefix.shape[2])
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=k_tree.device)
+    _check(load().longspec_hta_commit(ctypes.byref(dims), _ptr(k_prefix), _ptr(v_prefix),
+                                      _ptr(prefix_len), _ptr(k_tree), _ptr(v_tree),
+                                      _ptr(accept_len), _ptr(path), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)))
+
+
+def commit_paged(k_cache, v_cache, block_table, prefix_len, k_tree, v_tree, accept_len, path, *,
+                 L_cap, workspace=None, stream=None):
+    """commit() into a paged cache [num_blocks][Hkv][block_size][D]."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k_tree, "k_tree"), (v_tree, "v_tree")):
+        _need(t, n, torch.bfloat16, k_tree.device)
+    for t, n in ((block_table, "block_table"), (prefix_len, "prefix_len"), (accept_len, "accept_len"),
+                 (path, "path")):
+        _need(t, n, torch.int32, k_tree.device)
+    dims = _commit_dims(k_tree, L_cap)
+    kv = _paged(k_cache, v_cache, block_table, k_tree.device)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=k_tree.device)
+    _check(load().longspec_hta_commit_paged(ctypes.byref(dims), ctypes.byref(kv), _ptr(prefix_len),
+                                            _ptr(k_tree), _ptr(v_tree), _ptr(accept_len), _ptr(path),
+                                            _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def selftest_wait_timeout(workspace: torch.Tensor, stream=None) -> int:
