@@ -345,3 +345,18 @@ def commit_inputs(w: "Workload", seed: int, full_prefix: bool = False):
     inp["accept_len"] = torch.from_numpy(n)
     inp["path"] = torch.from_numpy(path)
     return inp
+
+
+def window_ring(k_ctx: torch.Tensor, v_ctx: torch.Tensor, prefix_lens, W: int):
+    """The last W positions of each sequence's context K/V [B][Hkv][L_max][D]
+    as a ring [B][Hkv][W][D]: position p at slot p mod W, for p in
+    [max(0, L_b - W), L_b); slots no position reaches are NaN (never read
+    as keys).  Pure data movement."""
+    B, Hkv, _, D = k_ctx.shape
+    k = torch.full((B, Hkv, W, D), float("nan"), dtype=k_ctx.dtype)
+    v = torch.full((B, Hkv, W, D), float("nan"), dtype=v_ctx.dtype)
+    for b, L in enumerate(int(x) for x in prefix_lens):
+        for p in range(max(0, L - W), L):
+            k[b, :, p % W] = k_ctx[b, :, p]
+            v[b, :, p % W] = v_ctx[b, :, p]
+    return k, v
