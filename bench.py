@@ -55,7 +55,8 @@ def workload_config(w, S, n_sets):
     if w.kind == "prefix":
         tree = "none (prefix-only attention)"
     lens = w.prefix_lens()
-    call = "longspec_hta_prefix_attention" if w.kind == "prefix" else "longspec_hta_verify"
+    call = {"prefix": "longspec_hta_prefix_attention",
+            "window": "longspec_hta_window_verify"}.get(w.kind, "longspec_hta_verify")
     if w.block_size:
         call += "_paged"
     return {"workload": w.name, "call": call, "block_size": w.block_size or None,
@@ -88,7 +89,7 @@ def prefix_algorithmic_bytes(w):
     """Bytes the prefix kernel must move at minimum: K and V of the L_b
     prefix keys of every (b, KV head) (2 * D * 2 bytes per key and head),
     plus Q once.  The split partials are not counted."""
-    lens = w.prefix_lens().astype(np.int64)
+    lens = w.visible_lens().astype(np.int64)
     return int(lens.sum()) * w.Hkv * 2 * w.D * 2 + w.B * w.Hq * w.T * w.D * 2
 
 
@@ -104,7 +105,7 @@ def floors(w, peak_gbs):
         tflops, sm_mhz = float(pk["bf16_tflops"]), float(pk.get("sm_max_mhz", 1965.0))
     except Exception:
         tflops, sm_mhz = 1590.0, 1965.0
-    keys = int(w.prefix_lens().astype(np.int64).sum()) * w.Hkv
+    keys = int(w.visible_lens().astype(np.int64).sum()) * w.Hkv
     rows = w.G * w.T
     padded = -(-rows // 128) * 128
     useful = 4.0 * rows * keys * w.D
@@ -225,6 +226,14 @@ def _oracle_head_problem(w, b, kvh):
     if key not in _ORACLE_CACHE:
         inp = w.generate_head(b, kvh)
         _ORACLE_CACHE.clear()
+        if w.kind == "window":
+            from oracle import window as oracle_window
+            args = [bf16_bits(inp["q"]), bf16_bits(inp["k_prefix"]), bf16_bits(inp["v_prefix"]),
+                    inp["prefix_len"].numpy(), bf16_bits(inp["k_tree"]), bf16_bits(inp["v_tree"]),
+                    inp["parent"].numpy()]
+            _ORACLE_CACHE[key] = lambda rows: oracle_window.window_attention(
+                *args, w.L_cap, scale=w.scale, rows=rows)
+            return _ORACLE_CACHE[key]
         _ORACLE_CACHE[key] = oracle.Problem(
             bf16_bits(inp["q"]), bf16_bits(inp["k_prefix"]), bf16_bits(inp["v_prefix"]),
             inp["prefix_len"].numpy(), bf16_bits(inp["k_tree"]), bf16_bits(inp["v_tree"]),
@@ -246,6 +255,8 @@ def oracle_rows_timed(w, heads, budget_s, rows_per_head=None, row_offset=0):
         t0 = time.perf_counter()
         if w.kind == "prefix":
             p.prefix_partial(0, w.L_cap, rows)
+        elif w.kind == "window":
+            p(rows)
         else:
             p.attention(rows)
         spent += time.perf_counter() - t0
@@ -320,6 +331,10 @@ def run_ours(args, world, rank, local):
     dims = hta.dims_of(base["q"], base["k_prefix"], w.scale)
     S, chunk = hta.chunking(dims, args.num_splits)
     ws = hta.new_workspace(dims, args.num_splits, dev)
+    if w.kind == "window":   # the window's W/128 + 1 tiles, split like a prefix of that length
+        span = hta.Dims(dims.B, dims.Hq, dims.Hkv, dims.D, dims.T, (w.L_cap // 128 + 1) * 128, dims.scale)
+        S, chunk = hta.chunking(span, 0)
+        ws = hta.new_window_workspace(dims, dev)
     out = torch.empty_like(base["q"])
     lse = torch.empty(base["q"].shape[:3], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -336,6 +351,14 @@ def run_ours(args, world, rank, local):
             hta.prefix_attention(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], out=out,
                                  lse=lse, workspace=ws, scale=w.scale, num_splits=args.num_splits,
                                  prefix_events=events, stream=stream)
+        elif w.kind == "window":
+            if events is not None:
+                events[0].record(stream)
+            hta.window_verify(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], s["k_tree"],
+                              s["v_tree"], s["parent"], out=out, lse=lse, workspace=ws,
+                              scale=w.scale, stream=stream)
+            if events is not None:    # around the whole call: no hook between its kernels
+                events[1].record(stream)
         else:
             hta.verify(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], s["k_tree"],
                        s["v_tree"], s["parent"], out=out, lse=lse, workspace=ws, scale=w.scale,
@@ -598,18 +621,21 @@ def run_e2e(args, w, cpu, dims, dev, stream, world):
             () if w.kind == "prefix" else ("k_tree", "v_tree", "parent"))
     elif w.kind == "prefix":
         names = ("q", "k_prefix", "v_prefix", "prefix_len")
+    elif w.kind == "window":
+        names = ("q", "k_prefix", "v_prefix", "prefix_len", "k_tree", "v_tree", "parent")
     else:
         names = tuple(cpu.keys())
     host = {k: cpu[k].pin_memory() for k in names}
     out = torch.empty_like(host["q"]).pin_memory()
     lse = torch.empty(host["q"].shape[:3], dtype=torch.float32).pin_memory()
-    if w.kind == "prefix" or w.block_size:
+    if w.kind in ("prefix", "window") or w.block_size:
         # no host-buffer entry point for these calls: the same copies in and
         # out around the device call, all on `stream`
         dsts = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
         dout = torch.empty_like(dsts["q"])
         dlse = torch.empty(dsts["q"].shape[:3], dtype=torch.float32, device=dev)
-        ws = hta.new_workspace(dims, args.num_splits, dev)
+        ws = (hta.new_window_workspace(dims, dev) if w.kind == "window"
+              else hta.new_workspace(dims, args.num_splits, dev))
 
         def device_call():
             s = dsts
@@ -619,6 +645,10 @@ def run_e2e(args, w, cpu, dims, dev, stream, world):
                 fn(s["q"], s["k_cache"], s["v_cache"], s["block_table"], s["prefix_len"], *tree,
                    L_cap=w.L_cap, out=dout, lse=dlse, workspace=ws, scale=w.scale,
                    num_splits=args.num_splits, stream=stream)
+            elif w.kind == "window":
+                hta.window_verify(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], s["k_tree"],
+                                  s["v_tree"], s["parent"], out=dout, lse=dlse, workspace=ws,
+                                  scale=w.scale, stream=stream)
             else:
                 hta.prefix_attention(s["q"], s["k_prefix"], s["v_prefix"], s["prefix_len"], out=dout,
                                      lse=dlse, workspace=ws, scale=w.scale,

@@ -339,6 +339,35 @@ LONGSPEC_HTA_API int longspec_hta_accept_greedy(int B, int T, int V, const void 
                                 int32_t *accept_len, int32_t *path, int32_t *bonus,
                                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Sliding-window tree attention: the draft model's self-attention while it
+ * drafts the tree.  LongSpec's draft model is one transformer block with
+ * sliding-window self-attention over 512 positions (LongSpec paper summary,
+ * "Summary"), so its own KV cache is a ring of W slots holding the last W
+ * positions, position p at slot p mod W.  A query at position p sees the W
+ * positions p - W + 1 .. p; a tree node at depth d (1 for parent -1) sits at
+ * position L_b + d - 1, so it sees its d ancestors-or-self and the context
+ * positions L_b + d - W .. L_b - 1 (clipped at 0):
+ *   dims: B, Hq, Hkv, D, T as in verify; L_cap = W, the ring size, a
+ *         multiple of 128 and > T (so a node's root path is in its window);
+ *   q bf16 [B][Hq][T][D]; k_ring/v_ring bf16 [B][Hkv][W][D];
+ *   prefix_len int32 [B]: the context length L_b >= 0 (it may exceed W);
+ *   k_tree/v_tree bf16 [B][Hkv][T][D], parent int32 [B][T] as in verify;
+ *   out bf16 [B][Hq][T][D], lse fp32 [B][Hq][T] (natural log);
+ *   workspace: longspec_hta_window_workspace_bytes(dims) bytes, 16-byte
+ *         aligned (status word first).
+ * Ring slots no position of the window maps to are never read as keys
+ * (they may hold anything).  Runs the tcgen05 prefix kernel over the window's
+ * tiles, split across CTAs like a prefix of W/128 + 1 tiles, and the tree
+ * pass + merge.  Errors: as verify, plus
+ * INVALID_DIMS for a W that is not a multiple of 128 or not above T; a
+ * negative prefix_len gives PREFIX_LEN_RANGE and NaN rows. */
+LONGSPEC_HTA_API size_t longspec_hta_window_workspace_bytes(const longspec_hta_dims *dims);
+LONGSPEC_HTA_API int longspec_hta_window_verify(const longspec_hta_dims *dims, const void *q,
+                                const void *k_ring, const void *v_ring, const int32_t *prefix_len,
+                                const void *k_tree, const void *v_tree, const int32_t *parent,
+                                void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
 /* Commit of the accepted path: after verification and acceptance, the
  * accepted tokens join the target's context, so their K/V rows (the tree
  * keys the verification pass used) are appended to the KV cache right after

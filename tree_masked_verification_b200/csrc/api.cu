@@ -614,6 +614,64 @@ int longspec_hta_accept_greedy(int B, int T, int V, const void *logits, const in
     return hta::launch_accept(p, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
 }
 
+// ---- sliding-window tree attention (the draft model's self-attention) ------
+namespace {
+// The window spans at most W/128 + 1 key tiles (its start need not be tile
+// aligned); they are split like a prefix of that many tiles.
+int window_tiles(const longspec_hta_dims *d) { return d->L_cap / hta::kKeyTile + 1; }
+
+Chunking window_chunking(const longspec_hta_dims *d, int num_sms) {
+    longspec_hta_dims span = *d;
+    span.L_cap = window_tiles(d) * hta::kKeyTile;
+    return chunking_for(&span, 0, num_sms);
+}
+
+int check_window_dims(const longspec_hta_dims *d) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (d->L_cap < 128 || d->L_cap % 128 != 0 || d->L_cap <= d->T) return LONGSPEC_HTA_ERR_INVALID_DIMS;
+    return LONGSPEC_HTA_OK;
+}
+}  // namespace
+
+size_t longspec_hta_window_workspace_bytes(const longspec_hta_dims *dims) {
+    if (check_window_dims(dims) != LONGSPEC_HTA_OK) return 0;
+    return ws_layout(dims, std::min(window_tiles(dims), hta::kMaxSplits)).total;
+}
+
+int longspec_hta_window_verify(const longspec_hta_dims *dims, const void *q, const void *k_ring,
+                               const void *v_ring, const int32_t *prefix_len, const void *k_tree,
+                               const void *v_tree, const int32_t *parent, void *out, float *lse,
+                               void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    int rc = check_window_dims(dims);
+    if (rc) return rc;
+    const int W = dims->L_cap;
+    const void *ptrs[] = {q, k_ring, v_ring, prefix_len, k_tree, v_tree, parent, out, lse, workspace};
+    for (const void *p : ptrs) {
+        if (!p) return LONGSPEC_HTA_ERR_NULL_POINTER;
+        if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
+    }
+    DeviceInfo di;
+    if ((rc = current_device(&di))) return rc;
+    const Chunking c = window_chunking(dims, di.num_sms);
+    const WsLayout w = ws_layout(dims, c.S);
+    if (workspace_bytes < w.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    float *o_part = reinterpret_cast<float *>(ws + w.o_off);
+    float *lse_part = reinterpret_cast<float *>(ws + w.lse_off);
+    PrefixParams pp = prefix_params(dims, c, q, k_ring, v_ring, prefix_len, o_part, lse_part, status);
+    pp.window = W;
+    pp.parent = parent;
+    if ((rc = run_prefix(dims, pp, LONGSPEC_HTA_PREFIX_TCGEN05, nullptr, nullptr, stream))) return rc;
+    TreeMergeParams tp = tree_params(dims, hta::kTreeModeMerge, c.S, q, k_tree, v_tree, parent, prefix_len,
+                                     o_part, lse_part, status);
+    tp.window = W;
+    tp.out = static_cast<__nv_bfloat16 *>(out);
+    tp.lse = lse;
+    return hta::launch_tree_merge(tp, stream) == cudaSuccess ? LONGSPEC_HTA_OK : LONGSPEC_HTA_ERR_CUDA;
+}
+
 // ---- KV commit of the accepted path ----------------------------------------
 namespace {
 int run_commit(const longspec_hta_dims *dims, void *k_cache, void *v_cache,

@@ -33,6 +33,7 @@ struct TreeMergeParams {
     float *o_tree, *lse_tree;         // kTreeModePartial outputs
     uint32_t *mask_out;               // kTreeModeMask output [B][T][ceil(T/32)]
     uint32_t *status;
+    int window;                       // > 0: sliding-window call, prefix_len may exceed L_cap
 };
 
 // Prefix split-KV partials.  Rows of one (b, KV head) are the packed query
@@ -52,6 +53,12 @@ struct PrefixParams {
     // and the tensor maps' boxes are block_size rows high.
     const int32_t *block_table;       // [B][max_blocks]
     int block_size, max_blocks, num_blocks;
+    // Sliding window (tcgen05 kernel only): window > 0 = the ring size W
+    // (= L_cap, a multiple of 128, > T); context position p sits at slot
+    // p mod W; a node at depth d sees positions [L_b + d - W, L_b).  The
+    // chunks cover the W/128 + 1 tiles from the one holding L_b - W.
+    int window;
+    const int32_t *parent;            // [B][T], for the depths (window only)
 };
 
 // Greedy (temperature-0) acceptance of a speculated tree.  logits bf16

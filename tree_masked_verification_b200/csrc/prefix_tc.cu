@@ -197,7 +197,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 }  // namespace
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool WINDOW>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const PrefixParams p) {
@@ -216,13 +216,14 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const size_t grow0 = static_cast<size_t>(bk) * p.M + row0;
     const float nan = __int_as_float(0x7fc00000);
     const int L = p.prefix_len[b];
-    if (L < 0 || L > p.L_cap) {
+    if (L < 0 || (!WINDOW && L > p.L_cap)) {
         if (threadIdx.x < C::BM && row0 + static_cast<int>(threadIdx.x) < p.M)
             p.lse_part[(grow0 + threadIdx.x) * p.S + split] = nan;
         if (threadIdx.x == 0) raise_status(p.status, kStatusPrefixLenRange);
         return;
     }
-    const int key_begin = split * p.chunk_tiles * C::BN;
+    // (sliding window: the chunks start at the tile holding L_b - W)
+    const int key_begin = (WINDOW ? max(0, L - p.window) / C::BN * C::BN : 0) + split * p.chunk_tiles * C::BN;
     const int key_end = min(L, key_begin + p.chunk_tiles * C::BN);
     const int n_tiles = key_end > key_begin ? (key_end - key_begin + C::BN - 1) / C::BN : 0;
     if (n_tiles == 0) {   // chunk past the end of this sequence: an empty partial
@@ -314,6 +315,25 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncwarp();
         return issued;
     };
+    // Producer of a K or V ring from the sliding-window ring cache (one
+    // thread): tile j holds context positions key_begin + j*128 + [0, 128),
+    // which sit at slots (key_begin + j*128) mod W + [0, 128) of this KV
+    // head's W-slot ring (W a multiple of 128, so a tile never wraps).
+    auto window_ring = [&](uint8_t *ring, const CUtensorMap *map, uint64_t *full, uint64_t *empty) {
+        int issued = 0;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j % C::NS;
+            if (*s_abort) break;
+            if (!mbar_wait(empty + st, ((j / C::NS) & 1) ^ 1)) { abort_cta(); break; }
+            uint8_t *stage = ring + st * C::KV_BYTES;
+            mbar_arrive_expect_tx(full + st, C::KV_BYTES);
+            const int y = bk * p.window + (key_begin + j * C::BN) % p.window;
+#pragma unroll
+            for (int h = 0; h < C::HALVES; ++h) tma_load_2d(stage + h * C::BOX_BYTES, map, full + st, h * 64, y);
+            issued = j + 1;
+        }
+        return issued;
+    };
     if (warp == kProducerKWarp) {
         // -------------------------------------------------------- TMA: Q, K
         regs_dec<kRegsOther>();
@@ -332,6 +352,15 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_wait(bars.q_full, 0);
                 for (int j = max(0, issued - C::NS); j < issued; ++j)
                     mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1);
+            }
+        } else if constexpr (WINDOW) {
+            if (lane == 0) {
+                const int issued = window_ring(smem + C::OFF_K, &tm_k, bars.k_full, bars.k_empty);
+                if (*s_abort) {
+                    mbar_wait(bars.q_full, 0);
+                    for (int j = max(0, issued - C::NS); j < issued; ++j)
+                        mbar_wait(bars.k_full + j % C::NS, (j / C::NS) & 1);
+                }
             }
         } else if (lane == 0) {
             int issued = 0;
@@ -363,6 +392,14 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (lane == 0 && *s_abort) {
                 for (int j = max(0, issued - C::NS); j < issued; ++j)
                     mbar_wait(bars.v_full + j % C::NS, (j / C::NS) & 1);
+            }
+        } else if constexpr (WINDOW) {
+            if (lane == 0) {
+                const int issued = window_ring(smem + C::OFF_V, &tm_v, bars.v_full, bars.v_empty);
+                if (*s_abort) {
+                    for (int j = max(0, issued - C::NS); j < issued; ++j)
+                        mbar_wait(bars.v_full + j % C::NS, (j / C::NS) & 1);
+                }
             }
         } else if (lane == 0) {
             int issued = 0;
@@ -488,6 +525,24 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float c2 = p.scale_log2;
         bool ok = true;
 
+        // sliding window: the first context position this row sees, L_b + d - W
+        // for its node's depth d (the parent walk is bounded; a bad parent
+        // array is reported by the tree pass, which writes the row as NaN)
+        int lo_row = 0;
+        if constexpr (WINDOW) {
+            const int rr = row0 + r;
+            if (rr < p.M) {
+                const int32_t *par = p.parent + static_cast<size_t>(b) * p.T;
+                int node = rr % p.T, d = 1;
+                for (int s = 0; s < p.T; ++s) {
+                    const int up = par[node];
+                    if (up < 0 || up >= node) break;
+                    node = up;
+                    ++d;
+                }
+                lo_row = L + d - p.window;
+            }
+        }
         float m_run = -INFINITY;      // running max of the scaled log2 scores (possibly stale)
         uint64_t l_exact = 0;         // pair of fp32 partial sums of 2^(x - m_run)
         uint64_t l_round = 0;         // the same over the bf16-rounded P that P*V uses
@@ -511,6 +566,20 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         r1[i] = (32 + i < n_valid) ? r1[i] : ninf;
                         r2[i] = (64 + i < n_valid) ? r2[i] : ninf;
                         r3[i] = (96 + i < n_valid) ? r3[i] : ninf;
+                    }
+                }
+                if constexpr (WINDOW) {
+                    // columns before this row's window (older than W - d positions)
+                    const int n_lo = lo_row - (key_begin + j * C::BN);
+                    if (n_lo > 0) {
+                        const uint32_t ninf = __float_as_uint(-INFINITY);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            r0[i] = (i < n_lo) ? ninf : r0[i];
+                            r1[i] = (32 + i < n_lo) ? ninf : r1[i];
+                            r2[i] = (64 + i < n_lo) ? ninf : r2[i];
+                            r3[i] = (96 + i < n_lo) ? ninf : r3[i];
+                        }
                     }
                 }
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -669,7 +738,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool WINDOW>
 cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                       const CUtensorMap &tm_v, cudaStream_t stream) {
     using C = TcCfg<D>;
@@ -680,7 +749,7 @@ cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUte
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(prefix_tc_kernel<D, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(prefix_tc_kernel<D, PAGED, WINDOW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_ALLOC);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
@@ -697,17 +766,20 @@ cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefix_tc_kernel<D, PAGED>, tm_q, tm_k, tm_v, p);
+    return cudaLaunchKernelEx(&cfg, prefix_tc_kernel<D, PAGED, WINDOW>, tm_q, tm_k, tm_v, p);
 }
 
 cudaError_t launch_prefix_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                              const CUtensorMap &tm_v, cudaStream_t stream) {
     const bool paged = p.block_table != nullptr;
+    if (p.window > 0)
+        return p.D == 128 ? launch_tc<128, false, true>(p, tm_q, tm_k, tm_v, stream)
+                          : launch_tc<64, false, true>(p, tm_q, tm_k, tm_v, stream);
     if (p.D == 128)
-        return paged ? launch_tc<128, true>(p, tm_q, tm_k, tm_v, stream)
-                     : launch_tc<128, false>(p, tm_q, tm_k, tm_v, stream);
-    return paged ? launch_tc<64, true>(p, tm_q, tm_k, tm_v, stream)
-                 : launch_tc<64, false>(p, tm_q, tm_k, tm_v, stream);
+        return paged ? launch_tc<128, true, false>(p, tm_q, tm_k, tm_v, stream)
+                     : launch_tc<128, false, false>(p, tm_q, tm_k, tm_v, stream);
+    return paged ? launch_tc<64, true, false>(p, tm_q, tm_k, tm_v, stream)
+                 : launch_tc<64, false, false>(p, tm_q, tm_k, tm_v, stream);
 }
 
 }  // namespace hta

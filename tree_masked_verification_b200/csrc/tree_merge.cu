@@ -128,7 +128,7 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
     // scheduled now: it waits for this grid before it reads anything.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int L = p.prefix_len[b];
-    const bool bad_len = L < 0 || L > p.L_cap;
+    const bool bad_len = L < 0 || (p.window == 0 && L > p.L_cap);
     if (bad_len && lane == 0 && rr == 0) raise_status(p.status, kStatusPrefixLenRange);
     float out_v[DPL];
     float lse_out;

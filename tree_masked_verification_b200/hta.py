@@ -49,7 +49,8 @@ EXPORTED = [
     "longspec_hta_selftest_wait_timeout", "longspec_hta_prefix_attention",
     "longspec_hta_verify_paged", "longspec_hta_prefix_attention_paged",
     "longspec_hta_accept_workspace_bytes", "longspec_hta_accept_greedy",
-    "longspec_hta_commit", "longspec_hta_commit_paged",
+    "longspec_hta_commit", "longspec_hta_commit_paged", "longspec_hta_window_verify",
+    "longspec_hta_window_workspace_bytes",
 ]
 
 
@@ -122,6 +123,9 @@ def load():
             lib.longspec_hta_accept_workspace_bytes.restype = sz
             lib.longspec_hta_accept_greedy.argtypes = [ci, ci, ci] + [vp] * 6 + [vp, sz, vp]
             lib.longspec_hta_commit.argtypes = [pd] + [vp] * 7 + [vp, sz, vp]
+            lib.longspec_hta_window_verify.argtypes = [pd] + [vp] * 9 + [vp, sz, vp]
+            lib.longspec_hta_window_workspace_bytes.argtypes = [pd]
+            lib.longspec_hta_window_workspace_bytes.restype = sz
             lib.longspec_hta_commit_paged.argtypes = [pd, pk] + [vp] * 5 + [vp, sz, vp]
             _lib = lib
     return _lib
@@ -422,6 +426,38 @@ def accept_greedy(logits, draft_tokens, parent, *, accept_len=None, path=None, b
         B, T, V, _ptr(logits), _ptr(draft_tokens), _ptr(parent), _ptr(accept_len), _ptr(path),
         _ptr(bonus), _ptr(workspace), workspace.numel(), _stream(stream)))
     return accept_len, path, bonus
+
+
+def new_window_workspace(dims: Dims, device=None) -> torch.Tensor:
+    n = int(load().longspec_hta_window_workspace_bytes(ctypes.byref(dims)))
+    if n == 0:
+        raise HtaError(ERR_INVALID_DIMS)
+    return torch.zeros(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def window_verify(q, k_ring, v_ring, prefix_len, k_tree, v_tree, parent, *, out=None, lse=None,
+                  workspace=None, scale: float = 0.0, stream=None):
+    """Sliding-window tree attention (the draft model's self-attention): the
+    ring k/v_ring [B][Hkv][W][D] holds context position p at slot p mod W;
+    a node at depth d sees its root path and positions [L_b + d - W, L_b)."""
+    _need(q, "q", torch.bfloat16)
+    dev = q.device
+    for t, n in ((k_ring, "k_ring"), (v_ring, "v_ring"), (k_tree, "k_tree"), (v_tree, "v_tree")):
+        _need(t, n, torch.bfloat16, dev)
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    _need(parent, "parent", torch.int32, dev)
+    dims = dims_of(q, k_ring, scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_window_workspace(dims, dev)
+    _check(load().longspec_hta_window_verify(
+        ctypes.byref(dims), _ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(prefix_len), _ptr(k_tree),
+        _ptr(v_tree), _ptr(parent), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out, lse
 
 
 def _commit_dims(k_tree, L_cap):

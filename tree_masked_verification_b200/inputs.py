@@ -101,6 +101,9 @@ class Workload:
     # tokens attend to the prefix alone (longspec_hta_prefix_attention, the
     # draft model's cross-attention into the target's KV cache)
     kind: str = "verify"
+    # "window": the draft model's sliding-window self-attention over the tree
+    # (longspec_hta_window_verify): k/v_prefix is the ring of W = L_cap slots
+    # and prefix_len the context length, which may exceed W
     # > 0: the prefix K/V in a paged cache of blocks of this many keys
     # (longspec_hta_verify_paged / _prefix_attention_paged)
     block_size: int = 0
@@ -115,6 +118,14 @@ class Workload:
         lo, hi = self.prefix_range
         g = _generator(self.seed, _S_LEN)
         return torch.randint(lo, hi + 1, (self.B,), generator=g).to(torch.int32).numpy()
+
+    def visible_lens(self) -> np.ndarray:
+        """Context keys a call must read per sequence: L_b, or for a
+        sliding-window call the min(L_b, W - 1) positions in some row's window."""
+        lens = self.prefix_lens()
+        if self.kind == "window":
+            return np.minimum(lens, self.L_cap - 1).astype(np.int32)
+        return lens
 
     def parents(self) -> np.ndarray:
         out = np.zeros((self.B, self.T), dtype=np.int32)
@@ -214,7 +225,7 @@ class Workload:
         """Bytes one call must move at minimum: prefix K+V of the L_b keys
         actually present, Q, tree K+V, out (bf16), lse (fp32), parent and
         prefix_len (int32)."""
-        lens = self.prefix_lens().astype(np.int64)
+        lens = self.visible_lens().astype(np.int64)
         kv = int(2 * self.Hkv * self.D * 2 * lens.sum())
         q = self.B * self.Hq * self.T * self.D * 2
         tree = 2 * self.B * self.Hkv * self.T * self.D * 2
@@ -252,6 +263,11 @@ WORKLOADS = {
     "draft-xattn-32k": Workload("draft-xattn-32k", B=1, Hq=32, Hkv=8, D=128,
                                 T=4, L_cap=32768, seed=6, tree="chain",
                                 kind="prefix"),
+    # the draft model's sliding-window (512) self-attention over the tree,
+    # 32k tokens of context, its K/V ring of 512 slots per KV head
+    "draft-window-512": Workload("draft-window-512", B=1, Hq=32, Hkv=8, D=128,
+                                 T=68, L_cap=512, seed=8, prefix_range=(32768, 32768),
+                                 kind="window"),
 }
 
 
