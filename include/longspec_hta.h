@@ -357,8 +357,8 @@ LONGSPEC_HTA_API int longspec_hta_accept_greedy(int B, int T, int V, const void 
  *         aligned (status word first).
  * Ring slots no position of the window maps to are never read as keys
  * (they may hold anything).  Runs the tcgen05 prefix kernel over the window's
- * tiles, split across CTAs like a prefix of W/128 + 1 tiles, and the tree
- * pass + merge.  Errors: as verify, plus
+ * W/128 + 1 tiles (one chunk per row tile and KV head) and the tree pass +
+ * merge.  Errors: as verify, plus
  * INVALID_DIMS for a W that is not a multiple of 128 or not above T; a
  * negative prefix_len gives PREFIX_LEN_RANGE and NaN rows. */
 LONGSPEC_HTA_API size_t longspec_hta_window_workspace_bytes(const longspec_hta_dims *dims);

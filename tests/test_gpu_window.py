@@ -58,8 +58,8 @@ CASES = {
     "longspec-tree": (1, 8, 2, 128, 68, [3001], 512, "levels"),
     "chain": (2, 2, 1, 64, 5, [600, 129], 128, "chain"),
     "empty-context": (2, 4, 2, 128, 7, [0, 40], 128, "random"),
-    # deep nodes whose window starts past the first key tile: with the
-    # window split across CTAs, their rows see no key in that tile's chunk
+    # deep nodes whose window starts past the first key tile: their rows see
+    # no key in that tile (a fully masked tile before the first real one)
     "deep-chain-wrapped": (1, 2, 1, 128, 40, [1000], 256, "chain"),
 }
 

@@ -526,8 +526,9 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool ok = true;
 
         // sliding window: the first context position this row sees, L_b + d - W
-        // for its node's depth d (the parent walk is bounded; a bad parent
-        // array is reported by the tree pass, which writes the row as NaN)
+        // for its node's depth d (the parent walk is bounded and overlaps the
+        // first tile's loads; a bad parent array is reported by the tree
+        // pass, which writes the row as NaN)
         int lo_row = 0;
         if constexpr (WINDOW) {
             const int rr = row0 + r;
