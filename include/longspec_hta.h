@@ -99,6 +99,9 @@ typedef struct {
 /* Prefix kernels selectable through longspec_hta_options.prefix_kernel. */
 #define LONGSPEC_HTA_PREFIX_TCGEN05 0   /* TMA + tcgen05/TMEM split-KV kernel (default) */
 #define LONGSPEC_HTA_PREFIX_SIMT    1   /* plain CUDA-core split-KV kernel, for cross-checks */
+#define LONGSPEC_HTA_PREFIX_TCGEN05_PAIR 2   /* tcgen05 kernel with two 128-row query tiles per
+                                                CTA when G*T > 128 (contiguous calls; others
+                                                run the default kernel); slower on B200 */
 
 /* Optional knobs of longspec_hta_verify_ex.  Zero-initialise for defaults. */
 typedef struct {
@@ -296,8 +299,8 @@ LONGSPEC_HTA_API int longspec_hta_prefix_attention(const longspec_hta_dims *dims
  * contiguous [B][Hkv][L_cap][D] arrays; every other argument, the result
  * and the error behaviour are the same.  The results equal those of the
  * contiguous call on the same keys bit for bit (same kernels, same split).
- * Only the tcgen05 prefix kernel reads a paged cache: prefix_kernel
- * LONGSPEC_HTA_PREFIX_SIMT returns LONGSPEC_HTA_ERR_INVALID_OPTION.  Host
+ * prefix_kernel LONGSPEC_HTA_PREFIX_SIMT returns
+ * LONGSPEC_HTA_ERR_INVALID_OPTION.  Host
  * errors: NULL_POINTER / MISALIGNED for the cache and table pointers,
  * INVALID_DIMS for a block_size not in {16, 32, 64, 128}, num_blocks < 1,
  * max_blocks * block_size < L_cap or a cache over 2^31 rows. */

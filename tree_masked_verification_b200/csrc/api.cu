@@ -141,12 +141,20 @@ int m_tiles_of(const longspec_hta_dims *d) {
     return (M + 127) / 128;
 }
 
+// With LONGSPEC_HTA_PREFIX_TCGEN05_PAIR, contiguous calls whose packed
+// group has more than 128 rows run two 128-row query tiles per CTA.
+bool pair_eligible(const longspec_hta_dims *d) { return (d->Hq / d->Hkv) * d->T > 128; }
+
+int cta_rows_units(const longspec_hta_dims *d, bool pair) {
+    return pair ? (m_tiles_of(d) + 1) / 2 : m_tiles_of(d);
+}
+
 // Split-KV chunking: chunk_tiles tiles of 128 keys per split, S splits.
 struct Chunking {
     int S, chunk_tiles;
 };
 
-Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms) {
+Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms, bool pair) {
     const int tiles = std::max(1, (d->L_cap + hta::kKeyTile - 1) / hta::kKeyTile);
     auto make = [&](int s) {
         s = std::max(1, std::min(std::min(s, tiles), hta::kMaxSplits));
@@ -155,7 +163,7 @@ Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms) {
     };
     if (requested > 0) return make(requested);
     // smallest estimated time: waves of CTAs x (tiles per CTA + fixed cost)
-    const long long units = 1LL * d->B * d->Hkv * m_tiles_of(d);
+    const long long units = 1LL * d->B * d->Hkv * cta_rows_units(d, pair);
     Chunking best = make(1);
     double best_cost = 1e300;
     for (int s = 1; s <= std::min(tiles, hta::kMaxSplits); ++s) {
@@ -207,7 +215,8 @@ PrefixParams prefix_params(const longspec_hta_dims *d, const Chunking &c, const 
 int run_prefix(const longspec_hta_dims *d, const PrefixParams &p, int kernel, cudaEvent_t ev_begin,
                cudaEvent_t ev_end, cudaStream_t stream) {
     CUtensorMap tq, tk, tv;
-    if (kernel == LONGSPEC_HTA_PREFIX_TCGEN05) {
+    const bool tc = kernel == LONGSPEC_HTA_PREFIX_TCGEN05 || kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR;
+    if (tc) {
         const uint64_t qrows = 1ull * d->B * d->Hq * d->T;
         const bool paged = p.block_table != nullptr;
         const uint64_t krows = paged ? 1ull * p.num_blocks * d->Hkv * p.block_size
@@ -219,9 +228,9 @@ int run_prefix(const longspec_hta_dims *d, const PrefixParams &p, int kernel, cu
         if ((rc = tensor_map(p.v_prefix, krows, d->D, &tv, box)) != LONGSPEC_HTA_OK) return rc;
     }
     if (ev_begin && cudaEventRecord(ev_begin, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
-    cudaError_t e = (kernel == LONGSPEC_HTA_PREFIX_TCGEN05)
-                        ? hta::launch_prefix_tc(p, tq, tk, tv, stream)
-                        : hta::launch_prefix_simt(p, stream);
+    PrefixParams pk = p;
+    pk.pair = kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR ? 1 : 0;
+    cudaError_t e = tc ? hta::launch_prefix_tc(pk, tq, tk, tv, stream) : hta::launch_prefix_simt(pk, stream);
     if (e != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
     if (ev_end && cudaEventRecord(ev_end, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
     return LONGSPEC_HTA_OK;
@@ -281,7 +290,7 @@ int longspec_hta_default_splits(const longspec_hta_dims *dims) {
     DeviceInfo di;
     rc = current_device(&di);
     if (rc) return rc;
-    return chunking_for(dims, 0, di.num_sms).S;
+    return chunking_for(dims, 0, di.num_sms, false).S;
 }
 
 int longspec_hta_chunking(const longspec_hta_dims *dims, int num_splits, int *num_splits_out,
@@ -295,7 +304,7 @@ int longspec_hta_chunking(const longspec_hta_dims *dims, int num_splits, int *nu
         if ((rc = current_device(&di))) return rc;
         sms = di.num_sms;
     }
-    const Chunking c = chunking_for(dims, num_splits, sms);
+    const Chunking c = chunking_for(dims, num_splits, sms, false);
     if (num_splits_out) *num_splits_out = c.S;
     if (chunk_keys_out) *chunk_keys_out = c.chunk_tiles * hta::kKeyTile;
     return LONGSPEC_HTA_OK;
@@ -309,7 +318,9 @@ size_t longspec_hta_workspace_bytes(const longspec_hta_dims *dims, int num_split
         if (current_device(&di) != LONGSPEC_HTA_OK) return 0;
         sms = di.num_sms;
     }
-    return ws_layout(dims, chunking_for(dims, num_splits, sms).S).total;
+    // large enough for either kernel's split count
+    const int S = std::max(chunking_for(dims, num_splits, sms, true).S, chunking_for(dims, num_splits, sms, false).S);
+    return ws_layout(dims, S).total;
 }
 
 int longspec_hta_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream) {
@@ -352,12 +363,14 @@ static int run_attention(const longspec_hta_dims *dims, const void *q, const voi
     longspec_hta_options o{};
     if (opts) o = *opts;
     if (o.num_splits < 0 || (o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
-                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT) ||
-        (kv && o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05))
+                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT &&
+                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05_PAIR) ||
+        (kv && o.prefix_kernel == LONGSPEC_HTA_PREFIX_SIMT))
         return LONGSPEC_HTA_ERR_INVALID_OPTION;
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
-    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms);
+    const bool pair = o.prefix_kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR && !kv && pair_eligible(dims);
+    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms, pair);
     const WsLayout w = ws_layout(dims, c.S);
     if (workspace_bytes < w.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -426,7 +439,7 @@ ArenaLayout arena_layout(const longspec_hta_dims *d, int num_sms) {
     a.par_b = 4ull * d->B * d->T;
     a.out_b = a.q_b;
     a.lse_b = 4ull * d->B * d->Hq * d->T;
-    a.ws_b = ws_layout(d, chunking_for(d, 0, num_sms).S).total;
+    a.ws_b = ws_layout(d, chunking_for(d, 0, num_sms, false).S).total;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align256(off + std::max<size_t>(bytes, 1)); return o; };
     a.q = take(a.q_b); a.kp = take(a.kv_b); a.vp = take(a.kv_b); a.plen = take(a.plen_b);
@@ -532,12 +545,14 @@ int longspec_hta_prefix_partial(const longspec_hta_dims *dims, const void *q, co
         if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
     }
     if (num_splits < 0 || (prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
-                           prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
+                           prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT &&
+                           prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05_PAIR))
         return LONGSPEC_HTA_ERR_INVALID_OPTION;
     if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
-    const Chunking c = chunking_for(dims, num_splits, di.num_sms);
+    const Chunking c = chunking_for(dims, num_splits, di.num_sms,
+                                    prefix_kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR && pair_eligible(dims));
     if (num_splits_out) *num_splits_out = c.S;
     const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part,
                                           static_cast<uint32_t *>(workspace));
@@ -819,9 +834,10 @@ extern "C" int longspec_hta_verify_noalloc(const longspec_hta_dims *dims, const 
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
     // the largest split count up to the usual choice whose partials fit
-    int S = chunking_for(dims, 0, di.num_sms).S;
-    while (S > 1 && ws_layout(dims, chunking_for(dims, S, di.num_sms).S).total > kNoAllocScratchBytes) --S;
-    const Chunking c = chunking_for(dims, S, di.num_sms);
+    const bool pair = false;
+    int S = chunking_for(dims, 0, di.num_sms, pair).S;
+    while (S > 1 && ws_layout(dims, chunking_for(dims, S, di.num_sms, pair).S).total > kNoAllocScratchBytes) --S;
+    const Chunking c = chunking_for(dims, S, di.num_sms, pair);
     const WsLayout w = ws_layout(dims, c.S);
     if (w.total > kNoAllocScratchBytes) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;

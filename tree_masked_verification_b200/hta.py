@@ -37,6 +37,7 @@ ERR_BAD_PATH = -21
 
 PREFIX_TCGEN05 = 0
 PREFIX_SIMT = 1
+PREFIX_TCGEN05_PAIR = 2     # tcgen05, two query tiles per CTA when G*T > 128 (slower)
 T_MAX = 256
 
 EXPORTED = [
@@ -372,6 +373,8 @@ def prefix_partial(q, k_prefix, v_prefix, prefix_len, *, scale: float = 0.0,
     (o_part fp32 [B][Hq][T][S][D], lse_part fp32 [B][Hq][T][S], chunk keys)."""
     dims = dims_of(q, k_prefix, scale)
     lib = load()
+    # the default call's split count, passed on explicitly so that every
+    # prefix kernel cuts the keys the same way
     S, chunk_keys = chunking(dims, num_splits)
     S_out = ctypes.c_int(0)
     B, Hq, T, D = q.shape
@@ -381,7 +384,7 @@ def prefix_partial(q, k_prefix, v_prefix, prefix_len, *, scale: float = 0.0,
         workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
     _check(lib.longspec_hta_prefix_partial(ctypes.byref(dims), _ptr(q), _ptr(k_prefix),
                                            _ptr(v_prefix), _ptr(prefix_len), _ptr(o), _ptr(l),
-                                           int(num_splits), int(prefix_kernel), ctypes.byref(S_out),
+                                           int(S), int(prefix_kernel), ctypes.byref(S_out),
                                            _ptr(workspace), workspace.numel(), _stream(stream)))
     if S_out.value != S:
         raise RuntimeError(f"split count mismatch: library {S_out.value}, binding {S}")
