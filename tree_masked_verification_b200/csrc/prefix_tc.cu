@@ -65,7 +65,7 @@ struct TcCfg {
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;    // slack to align the base to 1024
     // After the last MMA the K and V rings are free: the epilogue exchanges
-    // the groups' per-row statistics [group][m|l][row] in the
+    // the groups' per-row statistics [group][m|l_exact|l_round][row] in the
     // first K stage and stages the output rows [row][D] fp32 in the V ring.
     static constexpr int OFF_XCH = OFF_K;
     static constexpr int OFF_STAGE = OFF_V;
@@ -75,7 +75,7 @@ struct TcCfg {
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
     static_assert(COL_O + 2 * D <= TMEM_COLS, "tensor memory budget");
-    static_assert(2 * 2 * 128 * 4 <= KV_BYTES, "statistics exchange inside one K stage");
+    static_assert(2 * 3 * 128 * 4 <= KV_BYTES, "statistics exchange inside one K stage");
     static_assert(BM * D * 4 <= NS * KV_BYTES, "output staging inside the V ring");
 };
 
@@ -545,11 +545,8 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         float m_run = -INFINITY;      // running max of the scaled log2 scores (possibly stale)
-        // pair of fp32 partial sums of 2^(x - m_run), before P is rounded to
-        // bf16 for P*V: the rounding (relative 2^-9, to nearest) is unbiased,
-        // and keeping a second sum over the rounded P cost 2.4 us of the
-        // Llama-3-8B call in softmax issue slots
-        uint64_t l_exact = 0;
+        uint64_t l_exact = 0;         // pair of fp32 partial sums of 2^(x - m_run)
+        uint64_t l_round = 0;         // the same over the bf16-rounded P that P*V uses
         for (int j = grp, it = 0; j < n_tiles; j += 2, ++it) {
             if (ok && !warp_wait(bars.s_full + grp, it & 1)) { ok = false; abort_cta(); }
             tc_fence_after();
@@ -602,6 +599,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     alpha = ex2(m_run - m_new);              // 0 on the group's first tile
                     const uint64_t aa = f2(alpha, alpha);
                     l_exact = fma2(l_exact, aa, 0ull);
+                    l_round = fma2(l_round, aa, 0ull);
                     resc = it > 0;
                     m_run = m_new;
                 }
@@ -627,6 +625,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                         pk[k] = pack_bf16x2(p0, p1);
                         l_exact = add2(l_exact, f2(p0, p1));
+                        l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
                     }
                     tmem_st16(t_s + col, pk);
                 };
@@ -662,23 +661,25 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // merge the two groups' online softmaxes row by row (the lse merge
         // of two KV ranges): m = max(m_0, m_1), a_g = 2^(m_g - m),
         // O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1)
-        float *xch = reinterpret_cast<float *>(smem + C::OFF_XCH);   // [grp][m|l][row]
+        float *xch = reinterpret_cast<float *>(smem + C::OFF_XCH);   // [grp][m|le|lr][row]
         {
-            const float2 le = unf2(l_exact);
-            xch[(grp * 2 + 0) * 128 + r] = m_run;
-            xch[(grp * 2 + 1) * 128 + r] = le.x + le.y;
+            const float2 le = unf2(l_exact), lr = unf2(l_round);
+            xch[(grp * 3 + 0) * 128 + r] = m_run;
+            xch[(grp * 3 + 1) * 128 + r] = le.x + le.y;
+            xch[(grp * 3 + 2) * 128 + r] = lr.x + lr.y;
         }
         const bool failed = named_bar_or(1, 256, !ok || *s_abort);
-        const float m0 = xch[0 * 128 + r], m1 = xch[2 * 128 + r];
+        const float m0 = xch[0 * 128 + r], m1 = xch[3 * 128 + r];
         const float m = fmaxf(m0, m1);
         const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - m);
         const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - m);   // group 1 had no tile
-        const float l_ex = a0 * xch[1 * 128 + r] + a1 * xch[3 * 128 + r];
+        const float l_ex = a0 * xch[1 * 128 + r] + a1 * xch[4 * 128 + r];
+        const float l_rd = a0 * xch[2 * 128 + r] + a1 * xch[5 * 128 + r];
         const int rr = row0 + r;
         if (!failed) {
             // this group's half of the columns, normalised, into the staging
             // tile (16-byte chunks of a row XOR-swizzled by row % 8)
-            const float inv = 1.f / l_ex;
+            const float inv = 1.f / l_rd;
             const float c0 = a0 * inv, c1 = a1 * inv;
             const bool has1 = n_tiles > 1;
             float *stage = reinterpret_cast<float *>(smem + C::OFF_STAGE);
@@ -1024,7 +1025,7 @@ prefix_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const float c2 = p.scale_log2;
         bool ok = true;
         float m_run = -INFINITY;
-        uint64_t l_exact = 0;   // fp32 sums of 2^(x - m_run) before the bf16 rounding of P
+        uint64_t l_exact = 0, l_round = 0;
         if (grp < nq) {
             for (int j = 0; j < n_tiles; ++j) {
                 if (ok && !warp_wait(bars.s_full + grp, j & 1)) { ok = false; abort_cta(); }
@@ -1063,6 +1064,7 @@ prefix_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         alpha = ex2(m_run - m_new);              // 0 on the first tile
                         const uint64_t aa = f2(alpha, alpha);
                         l_exact = fma2(l_exact, aa, 0ull);
+                        l_round = fma2(l_round, aa, 0ull);
                         resc = j > 0;
                         m_run = m_new;
                     }
@@ -1086,6 +1088,7 @@ prefix_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                             pk[k] = pack_bf16x2(p0, p1);
                             l_exact = add2(l_exact, f2(p0, p1));
+                            l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
                         }
                         tmem_st16(t_s + col, pk);
                     };
@@ -1118,13 +1121,13 @@ prefix_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (ok && !warp_wait(bars.o_final, 0)) { ok = false; abort_cta(); }
             tc_fence_after();
             const bool failed = named_bar_or(1 + grp, 128, !ok || *s_abort);
-            const float2 le = unf2(l_exact);
-            const float l_ex = le.x + le.y;
+            const float2 le = unf2(l_exact), lr = unf2(l_round);
+            const float l_ex = le.x + le.y, l_rd = lr.x + lr.y;
             if (!failed) {
                 // normalised rows into the staging area (16-byte chunks of a
                 // row XOR-swizzled by row % 8), then a coalesced copy-out
                 float *stage = reinterpret_cast<float *>(smem + (grp == 0 ? C::OFF_K : C::OFF_V));
-                const float inv = 1.f / l_ex;
+                const float inv = 1.f / l_rd;
                 if (warp_active) {
 #pragma unroll 1
                     for (int c = 0; c < D; c += 32) {
