@@ -122,3 +122,10 @@ def test_rejects_misaligned_logits():
     with pytest.raises(hta.HtaError) as e:
         hta.accept_greedy(logits, d["draft_tokens"].cuda(), d["parent"].cuda())
     assert e.value.code == hta.ERR_MISALIGNED
+
+
+def test_many_sequences():
+    """64 sequences of the LongSpec tree (4 416 logits rows): one accept CTA
+    per sequence, slices spread over every row."""
+    d = accept_inputs(64, 68, 4096, 21, p_match=0.85)
+    _check(d["logits"], d["draft_tokens"], d["parent"], "B=64")

@@ -134,3 +134,42 @@ def test_bad_inputs_are_reported_and_leave_the_sequence(case):
     np.testing.assert_array_equal(_bits(d["kc"]), k)
     np.testing.assert_array_equal(_bits(d["vc"]), v)
     np.testing.assert_array_equal(d["prefix_len"].cpu().numpy(), new_len)
+
+
+@pytest.mark.parametrize("paged", [False, True], ids=["contiguous", "paged16"])
+def test_long_accepted_chain(paged):
+    """A 200-node chain accepted whole: 200 rows per KV head appended, across
+    many 16-key blocks."""
+    w = Workload("cm3", B=2, Hq=4, Hkv=2, D=128, T=200, L_cap=1200, seed=83, tree="chain",
+                 prefix_range=(100, 900))
+    inp = w.generate()
+    inp["accept_len"] = torch.tensor([200, 137], dtype=torch.int32)
+    inp["path"] = torch.tile(torch.arange(200, dtype=torch.int32), (2, 1))
+    inp["path"][1, 137:] = -1
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    if paged:
+        kc, vc, table = paged_cache(inp["k_prefix"], inp["v_prefix"], inp["prefix_len"].tolist(), 16,
+                                    seed=6, reserve=w.T)
+        d = _dev({"kc": kc, "vc": vc, "table": table, "prefix_len": inp["prefix_len"],
+                  "k_tree": inp["k_tree"], "v_tree": inp["v_tree"], "accept_len": inp["accept_len"],
+                  "path": inp["path"]})
+        hta.commit_paged(d["kc"], d["vc"], d["table"], d["prefix_len"], d["k_tree"], d["v_tree"],
+                         d["accept_len"], d["path"], L_cap=w.L_cap, workspace=ws)
+        k, v, new_len, errors = C.commit_paged(bf16_bits(kc), bf16_bits(vc), table.numpy(),
+                                               inp["prefix_len"].numpy(), bf16_bits(inp["k_tree"]),
+                                               bf16_bits(inp["v_tree"]), inp["accept_len"].numpy(),
+                                               inp["path"].numpy(), w.L_cap)
+        got_k, got_v = d["kc"], d["vc"]
+    else:
+        d = _dev(inp)
+        hta.commit(d["k_prefix"], d["v_prefix"], d["prefix_len"], d["k_tree"], d["v_tree"],
+                   d["accept_len"], d["path"], workspace=ws)
+        k, v, new_len, errors = C.commit(bf16_bits(inp["k_prefix"]), bf16_bits(inp["v_prefix"]),
+                                         inp["prefix_len"].numpy(), bf16_bits(inp["k_tree"]),
+                                         bf16_bits(inp["v_tree"]), inp["accept_len"].numpy(),
+                                         inp["path"].numpy())
+        got_k, got_v = d["k_prefix"], d["v_prefix"]
+    assert hta.get_status(ws) == hta.OK and not errors
+    np.testing.assert_array_equal(_bits(got_k), k)
+    np.testing.assert_array_equal(_bits(got_v), v)
+    np.testing.assert_array_equal(d["prefix_len"].cpu().numpy(), new_len)

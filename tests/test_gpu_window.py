@@ -61,6 +61,8 @@ CASES = {
     # deep nodes whose window starts past the first key tile: their rows see
     # no key in that tile (a fully masked tile before the first real one)
     "deep-chain-wrapped": (1, 2, 1, 128, 40, [1000], 256, "chain"),
+    # a 1024-slot ring (9 key tiles per call), four ragged contexts
+    "wide-ring-ragged": (4, 8, 2, 128, 20, [5000, 1024, 700, 2049], 1024, "random"),
 }
 
 
