@@ -28,6 +28,14 @@ class BadParent(ValueError):
     pass
 
 
+# Planted mistakes, used only by the pin-sensitivity test (None in all other
+# use): "ties-last" (argmax ties to the largest token), "own-row" (a node is
+# judged at the row after itself instead of its parent's), "shallowest"
+# (the shallowest accepted node wins), "bonus-root" (the bonus always comes
+# from the prefix-end row), "nan-wins" (NaN is not read as -inf).
+MUTATION = None
+
+
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """bf16 bit patterns (uint16) -> exact float64 values."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
@@ -37,7 +45,10 @@ def argmax_rows(logits_bits: np.ndarray) -> np.ndarray:
     """First index of the largest value of every row (bf16 bits, [..., V]),
     NaN read as -inf."""
     x = bf16_to_f64(logits_bits)
-    x = np.where(np.isnan(x), -np.inf, x)
+    if MUTATION != "nan-wins":
+        x = np.where(np.isnan(x), -np.inf, x)
+    if MUTATION == "ties-last":
+        return (x.shape[-1] - 1 - np.argmax(x[..., ::-1], axis=-1)).astype(np.int64)
     return np.argmax(x, axis=-1).astype(np.int64)
 
 
@@ -63,12 +74,21 @@ def accept_greedy(logits_bits: np.ndarray, draft_tokens: np.ndarray, parent: np.
         for i in range(T):                           # parents come first
             p = par[i]
             row = 0 if p == -1 else p + 1
+            if MUTATION == "own-row":
+                row = i + 1
             ok_parent = True if p == -1 else accepted[p]
             accepted[i] = ok_parent and int(draft_tokens[b][i]) == int(amax[b][row])
             depth[i] = 1 if p == -1 else depth[p] + 1
         best = -1
         for i in range(T):                           # deepest; the smallest id on ties
-            if accepted[i] and (best < 0 or depth[i] > depth[best]):
+            if not accepted[i]:
+                continue
+            if best < 0:
+                best = i
+            elif MUTATION == "shallowest":
+                if depth[i] < depth[best]:
+                    best = i
+            elif depth[i] > depth[best]:
                 best = i
         if best < 0:
             bonus[b] = amax[b][0]
@@ -81,5 +101,5 @@ def accept_greedy(logits_bits: np.ndarray, draft_tokens: np.ndarray, parent: np.
         chain.reverse()
         accept_len[b] = len(chain)
         path[b, :len(chain)] = chain
-        bonus[b] = amax[b][best + 1]
+        bonus[b] = amax[b][0 if MUTATION == "bonus-root" else best + 1]
     return accept_len, path, bonus

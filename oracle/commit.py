@@ -20,6 +20,13 @@ from __future__ import annotations
 import numpy as np
 
 
+# Planted mistakes, used only by the pin-sensitivity test (None in all other
+# use): "skip-one" (rows written one position late), "reversed" (the path
+# written leaf first), "no-advance" (prefix_len not advanced), "v-from-k"
+# (the V cache gets the tree K rows).
+MUTATION = None
+
+
 class CommitError(ValueError):
     def __init__(self, b: int, kind: str):
         super().__init__(f"sequence {b}: {kind}")
@@ -53,10 +60,11 @@ def commit(k_cache, v_cache, prefix_len, k_tree, v_tree, accept_len, path):
             continue
         for h in range(Hkv):
             for d in range(n):
-                node = int(path[b][d])
-                k[b, h, L + d] = k_tree[b, h, node]
-                v[b, h, L + d] = v_tree[b, h, node]
-        new_len[b] = L + n
+                node = int(path[b][n - 1 - d if MUTATION == "reversed" else d])
+                pos = L + d + (1 if MUTATION == "skip-one" and L + d + 1 < L_cap else 0)
+                k[b, h, pos] = k_tree[b, h, node]
+                v[b, h, pos] = (k_tree if MUTATION == "v-from-k" else v_tree)[b, h, node]
+        new_len[b] = L if MUTATION == "no-advance" else L + n
     return k, v, new_len, errors
 
 
@@ -78,10 +86,10 @@ def commit_paged(k_cache, v_cache, block_table, prefix_len, k_tree, v_tree, acce
             continue
         for h in range(Hkv):
             for d in range(n):
-                pos = L + d
+                pos = L + d + (1 if MUTATION == "skip-one" and L + d + 1 < L_cap else 0)
                 blk = int(block_table[b][pos // bs])
-                node = int(path[b][d])
+                node = int(path[b][n - 1 - d if MUTATION == "reversed" else d])
                 k[blk, h, pos % bs] = k_tree[b, h, node]
-                v[blk, h, pos % bs] = v_tree[b, h, node]
-        new_len[b] = L + n
+                v[blk, h, pos % bs] = (k_tree if MUTATION == "v-from-k" else v_tree)[b, h, node]
+        new_len[b] = L if MUTATION == "no-advance" else L + n
     return k, v, new_len, errors

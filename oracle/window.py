@@ -27,6 +27,13 @@ from __future__ import annotations
 import numpy as np
 
 
+# Planted mistakes, used only by the pin-sensitivity test (None in all other
+# use): "window+1" (one context key too many), "no-ring" (position p read at
+# slot p, not p mod W), "no-self" (a node does not see itself), "depth-0"
+# (depths counted from 0).
+MUTATION = None
+
+
 def _f64(bits) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -38,6 +45,8 @@ def depths(parent_b) -> list:
         if not (p == -1 or 0 <= p < i):
             raise ValueError(f"parent[{i}] = {p}")
         d.append(1 if p == -1 else d[p] + 1)
+    if MUTATION == "depth-0":
+        d = [x - 1 for x in d]
     return d
 
 
@@ -47,6 +56,8 @@ def ancestors_or_self(parent_b, t: int) -> list:
     while j != -1:
         out.append(j)
         j = int(parent_b[j])
+    if MUTATION == "no-self":
+        out.remove(t)
     return sorted(out)
 
 
@@ -76,9 +87,11 @@ def window_attention(q, k_ring, v_ring, prefix_len, k_tree, v_tree, parent, W: i
         L = int(prefix_len[b])
         d = dep[b][t]
         keys, vals = [], []
-        for p in range(max(0, L + d - W), L):              # context positions in the window
-            keys.append(krf[b, kvh, p % W])
-            vals.append(vrf[b, kvh, p % W])
+        first = L + d - W - (1 if MUTATION == "window+1" else 0)
+        for p in range(max(0, first), L):                  # context positions in the window
+            slot = min(p, W - 1) if MUTATION == "no-ring" else p % W
+            keys.append(krf[b, kvh, slot])
+            vals.append(vrf[b, kvh, slot])
         for j in ancestors_or_self(parent[b], t):          # the root path, itself included
             keys.append(ktf[b, kvh, j])
             vals.append(vtf[b, kvh, j])
