@@ -124,9 +124,94 @@ def pct(xs, q):
     return xs[min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))]
 
 
+def host_cpu():
+    """The host the CPU baseline ran on: logical CPUs available to this
+    process and the CPU model string."""
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except AttributeError:
+        nproc = os.cpu_count()
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": nproc, "cpu_model": model}
+
+
+class NvmlSampler:
+    """SM clock and throttle reasons read through NVML about every
+    `period_s` by a background thread, so that even a timed region of a
+    millisecond holds samples; only those stamped inside it are kept."""
+    NAMES = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+             ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, cuda_index, period_s=0.0005):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = None
+        try:
+            pr = torch.cuda.get_device_properties(cuda_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.period = period_s
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                bits = int(reasons_fn(h))
+            except Exception:
+                break
+            self.samples.append((time.time(), mhz, bits))
+            time.sleep(self.period)
+
+    def start(self):
+        self.thread.start()
+
+    def stop(self, t_begin=None, t_end=None):
+        self.stop_flag.set()
+        self.thread.join(timeout=2)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        inside = [r for r in self.samples if t_begin is not None and t_begin <= r[0] <= t_end]
+        use = inside or self.samples
+        if not use:
+            return None
+        reasons = sorted({n for _, _, bits in use for n, m in self.NAMES if bits & m})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": self.max_mhz,
+                "samples": len(use), "samples_in_timed_region": len(inside),
+                "reasons": reasons, "source": "NVML, ~0.5 ms period"}
+
+
+def clock_sampler(cuda_index):
+    try:
+        return NvmlSampler(cuda_index)
+    except Exception:
+        return ClockSampler(cuda_index)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms; only the
-    samples stamped inside the timed region are kept."""
+    samples stamped inside the timed region are kept (used when NVML cannot
+    be loaded)."""
     Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -175,7 +260,7 @@ class ClockSampler:
         reasons = set().union(*(r[3] for r in use))
         return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": use[-1][2],
                 "samples": len(use), "samples_in_timed_region": len(inside),
-                "reasons": sorted(reasons)}
+                "reasons": sorted(reasons), "source": "nvidia-smi, 200 ms period"}
 
 
 def dist_setup(n_gpus):
@@ -271,7 +356,7 @@ def cpu_baseline(w, budget_s=10.0):
     spent, rows = oracle_rows_timed(w, heads, budget_s)
     total_rows = w.B * w.Hq * w.T
     us_per_call = spent / rows * total_rows * 1e6
-    return {"value": us_per_call, "unit": "µs", "cores": 1, "kind": "oracle",
+    return {"value": us_per_call, "unit": "µs", "cores": 1, "kind": "oracle", **host_cpu(),
             "sample": f"{rows} of {total_rows} query rows (whole KV-head groups, fp64, one "
                       f"thread, {spent:.1f} s), scaled to one full call"}
 
@@ -302,7 +387,7 @@ def run_reference(args, world, rank):
         "ms_per_step": sec_per_row * per_step * 1e3, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, None, 1),
-        "cpu_baseline": {"value": us, "unit": "µs", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": us, "unit": "µs", "cores": 1, "kind": "oracle", **host_cpu(),
                          "sample": f"{per_step} query rows per step of {total_rows}, fp64, "
                                    f"one thread, scaled to one full call"},
         "e2e": {"value": us, "unit": "µs", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -389,7 +474,7 @@ def run_ours(args, world, rank, local):
 
     # timed region 1 (the headline): back-to-back calls, nothing between the
     # two kernels of a call (an event there would serialise them)
-    sampler = ClockSampler(local if world > 1 else 0)
+    sampler = clock_sampler(local if world > 1 else 0)
     sampler.start()
     time.sleep(0.3)
     t_start = torch.cuda.Event(enable_timing=True)
@@ -445,6 +530,8 @@ def run_ours(args, world, rank, local):
         call(i)
     host_us = (time.perf_counter() - h0) / n_host * 1e6
     torch.cuda.synchronize()
+    c_abi_us = c_abi_host_us(w, sets[0], out, lse, ws, dims, stream, n_host)
+    torch.cuda.synchronize()
 
     ms_per_step = elapsed_ms / args.steps
     us_per_call = job_us_per_call(elapsed_ms, args.steps, world)
@@ -478,6 +565,7 @@ def run_ours(args, world, rank, local):
             "prefix_us": {"p10": pct(prefix_ms, 0.1) * 1e3, "p50": pct(prefix_ms, 0.5) * 1e3,
                           "p90": pct(prefix_ms, 0.9) * 1e3},
             "host_api_us_per_call": host_us,
+            "c_abi_host_us_per_call": c_abi_us,
             "note": "per-call CUDA events of the roofline pass (events between the kernels "
                     "serialise them, so these run a little above the headline value)"},
         "floors": floors(w, peak),
@@ -536,7 +624,7 @@ def run_accept(args, world, rank, local):
         torch.cuda.synchronize()
         if hta.get_status(ws) != hta.OK:
             raise RuntimeError("device status error in the graph warm-up")
-    sampler = ClockSampler(local if world > 1 else 0)
+    sampler = clock_sampler(local if world > 1 else 0)
     sampler.start()
     time.sleep(0.3)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -652,9 +740,32 @@ def run_accept(args, world, rank, local):
             oracle_accept.accept_greedy(bits, tok, par)
             n += 1
         line["cpu_baseline"] = {"value": (time.perf_counter() - t_cpu) / n * 1e6, "unit": "µs",
-                                "cores": 1, "kind": "oracle",
+                                "cores": 1, "kind": "oracle", **host_cpu(),
                                 "sample": f"{n} whole calls of the numpy oracle on the same inputs"}
     print(json.dumps(line), flush=True)
+
+
+def c_abi_host_us(w, s, out, lse, ws, dims, stream, n):
+    """Host time of one longspec_hta_verify call on its own: the C entry
+    point called in a loop with its arguments converted once, so the figure
+    holds the library's checks, tensor-map lookups and launches but not the
+    Python binding's marshalling (the GPU runs behind).  None for calls other
+    than the contiguous verification."""
+    import ctypes
+    if w.kind != "verify" or w.block_size:
+        return None
+    fn = hta.load().longspec_hta_verify
+    args = (ctypes.byref(dims), s["q"].data_ptr(), s["k_prefix"].data_ptr(), s["v_prefix"].data_ptr(),
+            s["prefix_len"].data_ptr(), s["k_tree"].data_ptr(), s["v_tree"].data_ptr(),
+            s["parent"].data_ptr(), out.data_ptr(), lse.data_ptr(), ws.data_ptr(),
+            ws.numel(), stream.cuda_stream)
+    if fn(*args) != hta.OK:
+        raise RuntimeError("longspec_hta_verify failed")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        fn(*args)
+    return (time.perf_counter() - t0) / n * 1e6
 
 
 def run_e2e(args, w, cpu, dims, dev, stream, world):

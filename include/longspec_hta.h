@@ -99,9 +99,6 @@ typedef struct {
 /* Prefix kernels selectable through longspec_hta_options.prefix_kernel. */
 #define LONGSPEC_HTA_PREFIX_TCGEN05 0   /* TMA + tcgen05/TMEM split-KV kernel (default) */
 #define LONGSPEC_HTA_PREFIX_SIMT    1   /* plain CUDA-core split-KV kernel, for cross-checks */
-#define LONGSPEC_HTA_PREFIX_TCGEN05_PAIR 2   /* tcgen05 kernel with two 128-row query tiles per
-                                                CTA when G*T > 128 (contiguous calls; others
-                                                run the default kernel); slower on B200 */
 
 /* Optional knobs of longspec_hta_verify_ex.  Zero-initialise for defaults. */
 typedef struct {
@@ -200,9 +197,11 @@ LONGSPEC_HTA_API int longspec_hta_verify_ex(const longspec_hta_dims *dims,
  *   partials fit; a problem whose partials do not fit even with one split
  *   (B*Hq*T*(D+1)*4 bytes + 256 > 16 MiB) returns
  *   LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL and launches nothing.
- *   Set-up: the first call on each device looks up the array's device
- *   address (cudaGetSymbolAddress) with that device current; make that first
- *   call before any stream capture.
+ *   Set-up: the first call on each device, and the first call after the
+ *   current context on that device changed (a device reset, or a
+ *   driver-API context made current instead of the primary one), looks up
+ *   the array's device address (cudaGetSymbolAddress) in the current
+ *   context; make that first call before any stream capture.
  *   Sharing: every call on a device uses the same array.  Calls that can
  *   overlap on the GPU (different streams, or different host threads with no
  *   ordering between them) race on it and must be serialised by the caller.
@@ -216,6 +215,17 @@ LONGSPEC_HTA_API int longspec_hta_verify_noalloc(const longspec_hta_dims *dims,
                                 const void *k_tree, const void *v_tree,
                                 const int32_t *parent, void *out, float *lse,
                                 cudaStream_t stream);
+
+/*
+ * The split-KV chunking longspec_hta_verify_noalloc uses on a GPU with
+ * num_sms SMs (host only, no device needed): the split count
+ * longspec_hta_chunking would choose, lowered until the partials fit in the
+ * library's 16 MiB scratch.  Writes the split count and the keys per chunk;
+ * LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL when not even one split fits.  No
+ * counterpart in the pages.
+ */
+LONGSPEC_HTA_API int longspec_hta_noalloc_chunking(const longspec_hta_dims *dims, int num_sms,
+                                  int *num_splits_out, int *chunk_keys_out);
 
 /* Device bytes of the staging arena longspec_hta_verify_host needs: room
  * for every input and output plus the workspace, each 256-byte aligned. */

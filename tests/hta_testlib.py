@@ -2,11 +2,12 @@
 the parity gates.
 
 Gates (fp32 accumulation over bf16 inputs, out rounded to bf16):
-  * out: max |gpu - oracle| <= 1e-2 + h(oracle) and mean |gpu - oracle|
-    <= 1e-3, where h(x) is half the bf16 spacing at x: the result is
-    returned in bf16, and rounding the exact value alone moves it by up to
-    h(x) (0.0078 for |x| in [2, 4)), so the 1e-2 bound is applied to the
-    value before that final rounding;
+  * out: max |gpu - oracle| <= 1e-2 wherever |oracle| < 4, and mean
+    |gpu - oracle| <= 1e-3.  Where |oracle| >= 4 a bf16 output cannot meet
+    1e-2 by rounding alone (half the bf16 spacing there is 2^-6 = 0.0156 or
+    more), so there the bound is 1e-2 plus that half spacing h(oracle): the
+    1e-2 applies to the value before its final rounding.  Below 4 the half
+    spacing is at most 2^-7 = 0.0078 and no allowance is given;
   * lse: max |gpu - oracle| <= 1e-3 (natural log);
   * out, per row: ||gpu - oracle||_2 / ||oracle||_2 <= 2e-2.  The two
     absolute gates alone are blind at 32k keys, where |out| ~ 1e-2 and the
@@ -14,6 +15,9 @@ Gates (fp32 accumulation over bf16 inputs, out rounded to bf16):
     the separate tree-partial comparison are not.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -25,6 +29,12 @@ OUT_MAX_ABS = 1e-2
 OUT_MEAN_ABS = 1e-3
 LSE_ABS = 1e-3
 ROW_REL_L2 = 2e-2
+# below this magnitude a bf16 output gets no rounding allowance (half the
+# bf16 spacing is <= 2^-7 there)
+BF16_ALLOWANCE_FROM = 4.0
+# when set, every assert_parity call appends its margins (one JSON object
+# per line) to this file; the GPU suite's margins table is built from it
+PARITY_LOG = os.environ.get("HTA_PARITY_LOG")
 
 
 def to_device(inp: dict, device="cuda") -> dict:
@@ -53,8 +63,11 @@ def assert_parity(out, lse, out_ref, lse_ref, what=""):
     l_ref = np.asarray(lse_ref, dtype=np.float64).reshape(l.shape)
     assert np.isfinite(o).all() and np.isfinite(l).all(), f"{what}: non-finite output"
     d = np.abs(o - o_ref)
-    half_ulp = bf16_half_ulp(o_ref) if out.dtype == torch.bfloat16 else np.zeros_like(o_ref)
-    excess = d - (OUT_MAX_ABS + half_ulp)
+    if out.dtype == torch.bfloat16:
+        allowance = np.where(np.abs(o_ref) >= BF16_ALLOWANCE_FROM, bf16_half_ulp(o_ref), 0.0)
+    else:
+        allowance = np.zeros_like(o_ref)
+    excess = d - (OUT_MAX_ABS + allowance)
     D = o.shape[-1]
     rows_err = np.linalg.norm((o - o_ref).reshape(-1, D), axis=1)
     rows_ref = np.maximum(np.linalg.norm(o_ref.reshape(-1, D), axis=1), 1e-6)
@@ -62,12 +75,19 @@ def assert_parity(out, lse, out_ref, lse_ref, what=""):
     lse_err = np.abs(l - l_ref).max()
     msg = (f"{what}: out max {d.max():.3e} (over bound {excess.max():.3e}) mean {d.mean():.3e} "
            f"row-rel {rel:.3e} lse {lse_err:.3e}")
+    small = np.abs(o_ref) < BF16_ALLOWANCE_FROM
+    stats = dict(what=what, n=int(d.size), max_abs=float(d.max()), mean_abs=float(d.mean()),
+                 row_rel=float(rel), lse_abs=float(lse_err),
+                 max_abs_below4=float(d[small].max()) if small.any() else 0.0,
+                 max_abs_ref=float(np.abs(o_ref).max()), out_dtype=str(out.dtype))
+    if PARITY_LOG:
+        with open(PARITY_LOG, "a") as f:
+            f.write(json.dumps(stats) + "\n")
     assert excess.max() <= 0, msg
     assert d.mean() <= OUT_MEAN_ABS, msg
     assert lse_err <= LSE_ABS, msg
     assert rel <= ROW_REL_L2, msg
-    return dict(max_abs=float(d.max()), mean_abs=float(d.mean()), row_rel=float(rel),
-                lse_abs=float(lse_err))
+    return stats
 
 
 def sample_rows(w: Workload, n_heads: int = 3):

@@ -233,3 +233,45 @@ def test_commit_rejects_bad_arguments_on_host(lib):
     assert paged(hta.PagedKV(**{**base, "block_table": 0})) == hta.ERR_NULL_POINTER
     assert paged(hta.PagedKV(**{**base, "block_size": 24})) == hta.ERR_INVALID_DIMS
     assert paged(hta.PagedKV(**{**base, "max_blocks": 63})) == hta.ERR_INVALID_DIMS
+
+
+def _ws_bytes(d, S):
+    """Workspace bytes of S splits, written out from the layout the header
+    documents: 256-byte status region, O partials fp32 [rows][S][D], lse
+    partials fp32 [rows][S], each 256-byte aligned."""
+    a = lambda x: (x + 255) // 256 * 256
+    rows = d.B * d.Hq * d.T
+    return a(a(256 + rows * S * d.D * 4) + rows * S * 4)
+
+
+NOALLOC_SCRATCH = 16 << 20
+
+
+def test_noalloc_chunking_keeps_the_usual_split_when_it_fits(lib):
+    # Llama-3-8B shapes on 148 SMs: 6 splits of 43 tiles, 6.7 MB of partials
+    d = _dims()
+    assert hta.noalloc_chunking(d, 148) == (6, 43 * 128)
+    assert _ws_bytes(d, 6) <= NOALLOC_SCRATCH
+
+
+def test_noalloc_chunking_lowers_the_split_until_it_fits(lib):
+    # on a (hypothetical) 1024-SM part the usual choice would be 42 splits,
+    # 47 MB of partials: the call lowers it to the largest count that fits
+    d = _dims()
+    S, chunk = hta.noalloc_chunking(d, 1024)
+    assert _ws_bytes(d, S) <= NOALLOC_SCRATCH
+    tiles = 32768 // 128
+    assert (S - 1) * chunk < 32768 <= S * chunk
+    # every larger split count the chunking can produce does not fit
+    larger = {-(-tiles // -(-tiles // s)) for s in range(S + 1, 65)}
+    assert all(_ws_bytes(d, s) > NOALLOC_SCRATCH for s in larger if s > S)
+    assert S >= 10
+
+
+def test_noalloc_chunking_rejects_what_one_split_cannot_hold(lib):
+    # B*Hq*T*(D+1)*4 bytes of partials with one split: 67 MB > 16 MiB
+    d = _dims(B=8, Hq=64, T=256, L_cap=1024)
+    S, C = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib.longspec_hta_noalloc_chunking(ctypes.byref(d), 148, ctypes.byref(S), ctypes.byref(C))
+    assert rc == hta.ERR_WORKSPACE_TOO_SMALL
+    assert lib.longspec_hta_noalloc_chunking(ctypes.byref(_dims()), 0, None, None) == hta.ERR_INVALID_OPTION

@@ -50,8 +50,7 @@ SMALL = {
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
-@pytest.mark.parametrize("kernel", [hta.PREFIX_TCGEN05, hta.PREFIX_SIMT, hta.PREFIX_TCGEN05_PAIR],
-                         ids=["tc", "simt", "tc-pair"])
+@pytest.mark.parametrize("kernel", [hta.PREFIX_TCGEN05, hta.PREFIX_SIMT], ids=["tc", "simt"])
 @pytest.mark.parametrize("splits", [0, 1, 3])
 def test_verify_small_matches_oracle(name, kernel, splits):
     w = SMALL[name]
@@ -76,7 +75,7 @@ def test_prefix_partials_match_oracle_chunks(name, splits):
     cpu = w.generate()
     p = H.oracle_problem(cpu, w.scale)
     dev = H.to_device(cpu)
-    for kernel in (hta.PREFIX_TCGEN05, hta.PREFIX_SIMT, hta.PREFIX_TCGEN05_PAIR):
+    for kernel in (hta.PREFIX_TCGEN05, hta.PREFIX_SIMT):
         o, l, C = hta.prefix_partial(dev["q"], dev["k_prefix"], dev["v_prefix"],
                                      dev["prefix_len"], scale=w.scale, num_splits=splits,
                                      prefix_kernel=kernel)
@@ -207,7 +206,7 @@ def test_garbage_past_prefix_len_is_ignored():
         cpu["v_prefix"][b, :, lens[b]:] = float("inf")
     ref_out, ref_lse = H.oracle_problem(cpu).attention()
     dev = H.to_device(cpu)
-    for kernel in (hta.PREFIX_TCGEN05, hta.PREFIX_SIMT, hta.PREFIX_TCGEN05_PAIR):
+    for kernel in (hta.PREFIX_TCGEN05, hta.PREFIX_SIMT):
         out, lse = hta.verify(dev["q"], dev["k_prefix"], dev["v_prefix"], dev["prefix_len"],
                               dev["k_tree"], dev["v_tree"], dev["parent"], prefix_kernel=kernel)
         H.assert_parity(out, lse, ref_out, ref_lse, f"nan-tail/{kernel}")
@@ -275,8 +274,5 @@ def test_tc_matches_simt_at_llama_size():
                    dev["k_tree"], dev["v_tree"], dev["parent"], prefix_kernel=hta.PREFIX_TCGEN05)
     b = hta.verify(dev["q"], dev["k_prefix"], dev["v_prefix"], dev["prefix_len"],
                    dev["k_tree"], dev["v_tree"], dev["parent"], prefix_kernel=hta.PREFIX_SIMT)
-    c = hta.verify(dev["q"], dev["k_prefix"], dev["v_prefix"], dev["prefix_len"],
-                   dev["k_tree"], dev["v_tree"], dev["parent"], prefix_kernel=hta.PREFIX_TCGEN05_PAIR)
-    for x, y in ((a, b), (a, c)):
-        assert (x[0].float() - y[0].float()).abs().max() <= 1e-2
-        assert (x[1] - y[1]).abs().max() <= 1e-3
+    assert (a[0].float() - b[0].float()).abs().max() <= 1e-2
+    assert (a[1] - b[1]).abs().max() <= 1e-3

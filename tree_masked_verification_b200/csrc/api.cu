@@ -141,20 +141,12 @@ int m_tiles_of(const longspec_hta_dims *d) {
     return (M + 127) / 128;
 }
 
-// With LONGSPEC_HTA_PREFIX_TCGEN05_PAIR, contiguous calls whose packed
-// group has more than 128 rows run two 128-row query tiles per CTA.
-bool pair_eligible(const longspec_hta_dims *d) { return (d->Hq / d->Hkv) * d->T > 128; }
-
-int cta_rows_units(const longspec_hta_dims *d, bool pair) {
-    return pair ? (m_tiles_of(d) + 1) / 2 : m_tiles_of(d);
-}
-
 // Split-KV chunking: chunk_tiles tiles of 128 keys per split, S splits.
 struct Chunking {
     int S, chunk_tiles;
 };
 
-Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms, bool pair) {
+Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms) {
     const int tiles = std::max(1, (d->L_cap + hta::kKeyTile - 1) / hta::kKeyTile);
     auto make = [&](int s) {
         s = std::max(1, std::min(std::min(s, tiles), hta::kMaxSplits));
@@ -163,7 +155,7 @@ Chunking chunking_for(const longspec_hta_dims *d, int requested, int num_sms, bo
     };
     if (requested > 0) return make(requested);
     // smallest estimated time: waves of CTAs x (tiles per CTA + fixed cost)
-    const long long units = 1LL * d->B * d->Hkv * cta_rows_units(d, pair);
+    const long long units = 1LL * d->B * d->Hkv * m_tiles_of(d);
     Chunking best = make(1);
     double best_cost = 1e300;
     for (int s = 1; s <= std::min(tiles, hta::kMaxSplits); ++s) {
@@ -215,7 +207,7 @@ PrefixParams prefix_params(const longspec_hta_dims *d, const Chunking &c, const 
 int run_prefix(const longspec_hta_dims *d, const PrefixParams &p, int kernel, cudaEvent_t ev_begin,
                cudaEvent_t ev_end, cudaStream_t stream) {
     CUtensorMap tq, tk, tv;
-    const bool tc = kernel == LONGSPEC_HTA_PREFIX_TCGEN05 || kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR;
+    const bool tc = kernel == LONGSPEC_HTA_PREFIX_TCGEN05;
     if (tc) {
         const uint64_t qrows = 1ull * d->B * d->Hq * d->T;
         const bool paged = p.block_table != nullptr;
@@ -228,9 +220,7 @@ int run_prefix(const longspec_hta_dims *d, const PrefixParams &p, int kernel, cu
         if ((rc = tensor_map(p.v_prefix, krows, d->D, &tv, box)) != LONGSPEC_HTA_OK) return rc;
     }
     if (ev_begin && cudaEventRecord(ev_begin, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
-    PrefixParams pk = p;
-    pk.pair = kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR ? 1 : 0;
-    cudaError_t e = tc ? hta::launch_prefix_tc(pk, tq, tk, tv, stream) : hta::launch_prefix_simt(pk, stream);
+    cudaError_t e = tc ? hta::launch_prefix_tc(p, tq, tk, tv, stream) : hta::launch_prefix_simt(p, stream);
     if (e != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
     if (ev_end && cudaEventRecord(ev_end, stream) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
     return LONGSPEC_HTA_OK;
@@ -290,7 +280,7 @@ int longspec_hta_default_splits(const longspec_hta_dims *dims) {
     DeviceInfo di;
     rc = current_device(&di);
     if (rc) return rc;
-    return chunking_for(dims, 0, di.num_sms, false).S;
+    return chunking_for(dims, 0, di.num_sms).S;
 }
 
 int longspec_hta_chunking(const longspec_hta_dims *dims, int num_splits, int *num_splits_out,
@@ -304,7 +294,7 @@ int longspec_hta_chunking(const longspec_hta_dims *dims, int num_splits, int *nu
         if ((rc = current_device(&di))) return rc;
         sms = di.num_sms;
     }
-    const Chunking c = chunking_for(dims, num_splits, sms, false);
+    const Chunking c = chunking_for(dims, num_splits, sms);
     if (num_splits_out) *num_splits_out = c.S;
     if (chunk_keys_out) *chunk_keys_out = c.chunk_tiles * hta::kKeyTile;
     return LONGSPEC_HTA_OK;
@@ -318,9 +308,7 @@ size_t longspec_hta_workspace_bytes(const longspec_hta_dims *dims, int num_split
         if (current_device(&di) != LONGSPEC_HTA_OK) return 0;
         sms = di.num_sms;
     }
-    // large enough for either kernel's split count
-    const int S = std::max(chunking_for(dims, num_splits, sms, true).S, chunking_for(dims, num_splits, sms, false).S);
-    return ws_layout(dims, S).total;
+    return ws_layout(dims, chunking_for(dims, num_splits, sms).S).total;
 }
 
 int longspec_hta_workspace_init(void *workspace, size_t workspace_bytes, cudaStream_t stream) {
@@ -363,14 +351,12 @@ static int run_attention(const longspec_hta_dims *dims, const void *q, const voi
     longspec_hta_options o{};
     if (opts) o = *opts;
     if (o.num_splits < 0 || (o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
-                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT &&
-                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05_PAIR) ||
+                             o.prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT) ||
         (kv && o.prefix_kernel == LONGSPEC_HTA_PREFIX_SIMT))
         return LONGSPEC_HTA_ERR_INVALID_OPTION;
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
-    const bool pair = o.prefix_kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR && !kv && pair_eligible(dims);
-    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms, pair);
+    const Chunking c = chunking_for(dims, o.num_splits, di.num_sms);
     const WsLayout w = ws_layout(dims, c.S);
     if (workspace_bytes < w.total) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -439,7 +425,7 @@ ArenaLayout arena_layout(const longspec_hta_dims *d, int num_sms) {
     a.par_b = 4ull * d->B * d->T;
     a.out_b = a.q_b;
     a.lse_b = 4ull * d->B * d->Hq * d->T;
-    a.ws_b = ws_layout(d, chunking_for(d, 0, num_sms, false).S).total;
+    a.ws_b = ws_layout(d, chunking_for(d, 0, num_sms).S).total;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align256(off + std::max<size_t>(bytes, 1)); return o; };
     a.q = take(a.q_b); a.kp = take(a.kv_b); a.vp = take(a.kv_b); a.plen = take(a.plen_b);
@@ -545,14 +531,12 @@ int longspec_hta_prefix_partial(const longspec_hta_dims *dims, const void *q, co
         if (!aligned16(p)) return LONGSPEC_HTA_ERR_MISALIGNED;
     }
     if (num_splits < 0 || (prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05 &&
-                           prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT &&
-                           prefix_kernel != LONGSPEC_HTA_PREFIX_TCGEN05_PAIR))
+                           prefix_kernel != LONGSPEC_HTA_PREFIX_SIMT))
         return LONGSPEC_HTA_ERR_INVALID_OPTION;
     if (workspace_bytes < static_cast<size_t>(hta::kStatusBytes)) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
-    const Chunking c = chunking_for(dims, num_splits, di.num_sms,
-                                    prefix_kernel == LONGSPEC_HTA_PREFIX_TCGEN05_PAIR && pair_eligible(dims));
+    const Chunking c = chunking_for(dims, num_splits, di.num_sms);
     if (num_splits_out) *num_splits_out = c.S;
     const PrefixParams pp = prefix_params(dims, c, q, k_prefix, v_prefix, prefix_len, o_part, lse_part,
                                           static_cast<uint32_t *>(workspace));
@@ -797,27 +781,83 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void *g_noalloc_ptr[kMaxDevices];
+// The array's address belongs to the context the module was loaded in:
+// after a device reset, or with another context current on the same device
+// (a driver-API context instead of the primary one), the module is loaded
+// again, possibly elsewhere.  So the cached address is keyed on the current
+// context as well as the device, and looked up again when that changes.
+struct NoAllocSlot {
+    CUcontext ctx;
+    void *ptr;
+};
+NoAllocSlot g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Device address of the static scratch on the current device: set up once
-// per device (cudaGetSymbolAddress, a query, not an allocation).  In host
-// code the array's name only stands in for it and must never reach a kernel.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Device address of the static scratch in the current context
+// (cudaGetSymbolAddress, a query, not an allocation).  In host code the
+// array's name only stands in for it and must never reach a kernel.
 int noalloc_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LONGSPEC_HTA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return LONGSPEC_HTA_ERR_UNSUPPORTED_DEVICE;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return LONGSPEC_HTA_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return LONGSPEC_HTA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoAllocSlot &slot = g_noalloc[dev];
+    if (!slot.ptr || !ctx || slot.ctx != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LONGSPEC_HTA_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        // the lookup makes the device's primary context current if none was
+        if (!ctx && get_ctx(&ctx) != CUDA_SUCCESS) return LONGSPEC_HTA_ERR_CUDA;
+        slot.ctx = ctx;
+        slot.ptr = p;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return LONGSPEC_HTA_OK;
 }
 
+// The split-KV chunking the no-allocation call uses on a GPU with `num_sms`
+// SMs: the usual choice, or the largest smaller split count whose partials
+// fit in the static scratch.  ok = false: not even one split fits.
+Chunking noalloc_chunking(const longspec_hta_dims *dims, int num_sms, bool *ok) {
+    int S = chunking_for(dims, 0, num_sms).S;
+    while (S > 1 && ws_layout(dims, chunking_for(dims, S, num_sms).S).total > kNoAllocScratchBytes) --S;
+    const Chunking c = chunking_for(dims, S, num_sms);
+    *ok = ws_layout(dims, c.S).total <= kNoAllocScratchBytes;
+    return c;
+}
+
 }  // namespace
+
+extern "C" int longspec_hta_noalloc_chunking(const longspec_hta_dims *dims, int num_sms,
+                                             int *num_splits_out, int *chunk_keys_out) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (num_sms < 1) return LONGSPEC_HTA_ERR_INVALID_OPTION;
+    bool ok = false;
+    const Chunking c = noalloc_chunking(dims, num_sms, &ok);
+    if (!ok) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
+    if (num_splits_out) *num_splits_out = c.S;
+    if (chunk_keys_out) *chunk_keys_out = c.chunk_tiles * hta::kKeyTile;
+    return LONGSPEC_HTA_OK;
+}
 
 extern "C" int longspec_hta_verify_noalloc(const longspec_hta_dims *dims, const void *q,
                                            const void *k_prefix, const void *v_prefix,
@@ -834,12 +874,10 @@ extern "C" int longspec_hta_verify_noalloc(const longspec_hta_dims *dims, const 
     DeviceInfo di;
     if ((rc = current_device(&di))) return rc;
     // the largest split count up to the usual choice whose partials fit
-    const bool pair = false;
-    int S = chunking_for(dims, 0, di.num_sms, pair).S;
-    while (S > 1 && ws_layout(dims, chunking_for(dims, S, di.num_sms, pair).S).total > kNoAllocScratchBytes) --S;
-    const Chunking c = chunking_for(dims, S, di.num_sms, pair);
+    bool fits = false;
+    const Chunking c = noalloc_chunking(dims, di.num_sms, &fits);
+    if (!fits) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     const WsLayout w = ws_layout(dims, c.S);
-    if (w.total > kNoAllocScratchBytes) return LONGSPEC_HTA_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;
     if ((rc = noalloc_scratch(&scratch))) return rc;
     uint8_t *ws = static_cast<uint8_t *>(scratch);

@@ -59,9 +59,6 @@ struct PrefixParams {
     // chunks cover the W/128 + 1 tiles from the one holding L_b - W.
     int window;
     const int32_t *parent;            // [B][T], for the depths (window only)
-    // 1: contiguous calls with M > 128 run two query tiles per CTA
-    // (prefix_pair_kernel); 0: one query tile per CTA
-    int pair;
 };
 
 // Greedy (temperature-0) acceptance of a speculated tree.  logits bf16

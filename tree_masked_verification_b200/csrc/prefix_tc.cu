@@ -739,468 +739,6 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
-// ---------------------------------------------------------------------------
-// Paired query tiles (LONGSPEC_HTA_PREFIX_TCGEN05_PAIR; not the default: on
-// B200 it ran at the same time per 128-row tile as the kernel above, so the
-// extra padding of 256-row CTAs made the Llama-3-8B call slower, 74.5 against
-// 62.7 us).  When the packed group has more than 128 rows (G*T > 128: 272
-// for Llama-3-8B's 32/8 heads and the 68-node tree), one CTA takes two
-// 128-row query tiles over the same K/V chunk, one softmax warpgroup per
-// tile.  The MMA issuer interleaves the tiles, so while one group computes
-// the exponentials of tile j the tensor pipe runs the other group's P*V and
-// Q*K^T: the per-tile chain of one group (softmax, then P V_j and Q K_{j+1}^T)
-// overlaps the other's, and each K/V tile read from shared memory serves
-// 256 rows.  Tensor memory: S[g] (128 columns) and O[g] (D columns) per query
-// tile g, 512 columns in all; each group's online softmax covers every key
-// tile of the chunk, so no merge between the groups is needed.  A CTA whose
-// second tile holds no row runs the first tile alone.
-template <int D>
-struct PairCfg {
-    static constexpr int BM = 128;                          // rows per query tile
-    static constexpr int BN = kKeyTile;
-    static constexpr int NSK = (D == 128) ? 3 : 4;          // K ring depth
-    static constexpr int NSV = (D == 128) ? 2 : 4;          // V ring depth
-    static constexpr int HALVES = D / 64;
-    static constexpr int BOX_BYTES = 128 * 64 * 2;
-    static constexpr int QT_BYTES = BM * D * 2;             // one query tile
-    static constexpr int KV_BYTES = BN * D * 2;
-    static constexpr int OFF_Q = 0;                         // tile g at OFF_Q + g * QT_BYTES
-    static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
-    static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
-    static constexpr int NUM_BARS = 1 + 2 * NSK + 2 * NSV + 1 + 2 + 2 + 2;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_MISC + 16;
-    static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-    // after the last MMA, group g stages its output rows [row][D] fp32 in
-    // the K ring (g = 0) or the V ring (g = 1)
-    static constexpr int TMEM_COLS = 512;
-    static constexpr int COL_S = 0;
-    static constexpr int COL_O = 256;
-    static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
-    static_assert(COL_O + 2 * D <= TMEM_COLS, "tensor memory budget");
-    static_assert(BM * D * 4 <= NSV * KV_BYTES && NSV <= NSK, "output staging inside one ring");
-    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-};
-
-template <int D>
-__global__ void __launch_bounds__(kThreadsTc, 1)
-prefix_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefixParams p) {
-    using C = PairCfg<D>;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mt = blockIdx.x, split = blockIdx.y, bk = blockIdx.z;
-    const int b = bk / p.Hkv;
-    const int row0 = mt * 2 * C::BM;                        // first row of query tile 0
-    const int nq = (row0 + C::BM < p.M) ? 2 : 1;            // query tiles holding rows
-    const size_t grow0 = static_cast<size_t>(bk) * p.M + row0;
-    const float nan = __int_as_float(0x7fc00000);
-    const int L = p.prefix_len[b];
-    if (L < 0 || L > p.L_cap) {
-        for (int i = threadIdx.x; i < nq * C::BM; i += blockDim.x)
-            if (row0 + i < p.M) p.lse_part[(grow0 + i) * p.S + split] = nan;
-        if (threadIdx.x == 0) raise_status(p.status, kStatusPrefixLenRange);
-        return;
-    }
-    const int key_begin = split * p.chunk_tiles * C::BN;
-    const int key_end = min(L, key_begin + p.chunk_tiles * C::BN);
-    const int n_tiles = key_end > key_begin ? (key_end - key_begin + C::BN - 1) / C::BN : 0;
-    if (n_tiles == 0) {
-        for (int i = threadIdx.x; i < nq * C::BM; i += blockDim.x)
-            if (row0 + i < p.M) p.lse_part[(grow0 + i) * p.S + split] = -INFINITY;
-        return;
-    }
-    const int last_valid = key_end - (key_begin + (n_tiles - 1) * C::BN);   // 1..128
-
-    Bars bars;
-    {
-        uint64_t *base = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-        bars.q_full = base;
-        bars.k_full = base + 1;
-        bars.k_empty = bars.k_full + C::NSK;
-        bars.v_full = bars.k_empty + C::NSK;
-        bars.v_empty = bars.v_full + C::NSV;
-        bars.v_tail = bars.v_empty + C::NSV;
-        bars.s_full = bars.v_tail + 1;
-        bars.p_ready = bars.s_full + 2;
-        bars.o_final = bars.p_ready + 2;
-        bars.drain = bars.o_final + 1;
-    }
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-    if (threadIdx.x == 0) {
-        mbar_init(bars.q_full, 1);
-        for (int i = 0; i < C::NSK; ++i) {
-            mbar_init(bars.k_full + i, 1);
-            mbar_init(bars.k_empty + i, 1);
-        }
-        for (int i = 0; i < C::NSV; ++i) {
-            mbar_init(bars.v_full + i, 1);
-            mbar_init(bars.v_empty + i, 1);
-        }
-        mbar_init(bars.v_tail, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bars.s_full + i, 1);
-            mbar_init(bars.p_ready + i, 4);
-        }
-        mbar_init(bars.o_final, 1);
-        mbar_init(bars.drain, 1);
-        *s_abort = 0;
-        fence_barrier_init();
-    }
-    if (warp == kMmaWarp) {
-        tmem_alloc(s_tmem, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-    auto abort_cta = [&]() {
-        *s_abort = 1;
-        raise_status(p.status, kStatusPipelineTimeout);
-    };
-    const int kv_row0 = bk * p.L_cap + key_begin;
-    if (warp == kProducerKWarp) {
-        // ----------------------------------------------------- TMA: Q, K
-        regs_dec<kRegsOther>();
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            mbar_arrive_expect_tx(bars.q_full, nq * C::QT_BYTES);
-            for (int g = 0; g < nq; ++g)
-#pragma unroll
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_2d(smem + C::OFF_Q + g * C::QT_BYTES + h * C::BOX_BYTES, &tm_q, bars.q_full,
-                                h * 64, static_cast<int>(grow0) + g * C::BM);
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int st = j % C::NSK;
-                if (*s_abort) break;
-                if (!mbar_wait(bars.k_empty + st, ((j / C::NSK) & 1) ^ 1)) { abort_cta(); break; }
-                uint8_t *sk = smem + C::OFF_K + st * C::KV_BYTES;
-                mbar_arrive_expect_tx(bars.k_full + st, C::KV_BYTES);
-#pragma unroll
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_2d(sk + h * C::BOX_BYTES, &tm_k, bars.k_full + st, h * 64, kv_row0 + j * C::BN);
-                issued = j + 1;
-            }
-            if (*s_abort) {
-                mbar_wait(bars.q_full, 0);
-                for (int j = max(0, issued - C::NSK); j < issued; ++j)
-                    mbar_wait(bars.k_full + j % C::NSK, (j / C::NSK) & 1);
-            }
-        }
-        __syncwarp();
-    } else if (warp == kProducerVWarp) {
-        // ----------------------------------------------------------- TMA: V
-        regs_dec<kRegsOther>();
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_v);
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int st = j % C::NSV;
-                if (*s_abort) break;
-                if (!mbar_wait(bars.v_empty + st, ((j / C::NSV) & 1) ^ 1)) { abort_cta(); break; }
-                uint8_t *sv = smem + C::OFF_V + st * C::KV_BYTES;
-                mbar_arrive_expect_tx(bars.v_full + st, C::KV_BYTES);
-#pragma unroll
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_2d(sv + h * C::BOX_BYTES, &tm_v, bars.v_full + st, h * 64, kv_row0 + j * C::BN);
-                issued = j + 1;
-            }
-            if (*s_abort) {
-                for (int j = max(0, issued - C::NSV); j < issued; ++j)
-                    mbar_wait(bars.v_full + j % C::NSV, (j / C::NSV) & 1);
-            }
-        }
-        __syncwarp();
-        if (last_valid < C::BN) {
-            // rows past L_b of the last V tile may hold anything: zero them
-            const int j = n_tiles - 1;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(bars.v_full + j % C::NSV, (j / C::NSV) & 1));
-            if (ok) {
-                uint8_t *sv = smem + C::OFF_V + (j % C::NSV) * C::KV_BYTES;
-                const int per_row = C::HALVES * 8;
-                for (int idx = lane; idx < (C::BN - last_valid) * per_row; idx += 32) {
-                    const int r = last_valid + idx / per_row;
-                    const int h = (idx % per_row) / 8, c = idx % 8;
-                    *reinterpret_cast<uint4 *>(sv + h * C::BOX_BYTES + r * 128 + c * 16) =
-                        make_uint4(0u, 0u, 0u, 0u);
-                }
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bars.v_tail);
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA
-        regs_dec<kRegsOther>();
-        // Order: QK(0,0) QK(1,0), then per key tile j and query tile g:
-        // [PV(g,j), QK(g,j+1)].  QK(g,j+1) overwrites S[g], whose P is read
-        // by PV(g,j) just before it in issue order.  K_j is released after
-        // the last query tile's QK of it, V_j after the last PV of it.
-        if (lane == 0) {
-            const uint32_t sk0 = smem_u32(smem + C::OFF_K), sv0 = smem_u32(smem + C::OFF_V);
-            const uint64_t kdesc0 = smem_desc_sw128(sk0, 16, 1024);
-            const uint64_t vdesc0 = smem_desc_sw128(sv0, C::BOX_BYTES, 1024);
-            auto issue_qk = [=](int g, int j) {
-                const int st = j % C::NSK;
-                const uint64_t qd = smem_desc_sw128(smem_u32(smem + C::OFF_Q + g * C::QT_BYTES), 16, 1024);
-                const uint64_t kd = kdesc0 + ((st * C::KV_BYTES) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + C::COL_S + g * 128, qd + (off >> 4), kd + (off >> 4), C::IDESC_QK,
-                           kk > 0 ? 1u : 0u);
-                }
-                if (g == nq - 1) mma_commit(bars.k_empty + st);
-                mma_commit(bars.s_full + g);
-            };
-            auto issue_pv = [=](int g, int j) {
-                const int st = j % C::NSV;
-                const uint64_t vd = vdesc0 + ((st * C::KV_BYTES) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ts(tmem + C::COL_O + g * D, tmem + C::COL_S + g * 128 + kk * 8,
-                           vd + ((kk * 16 * 128) >> 4), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-                if (g == nq - 1) {
-                    mma_commit(bars.v_empty + st);
-                    if (j == n_tiles - 1) mma_commit(bars.o_final);
-                }
-            };
-            bool ok = mbar_wait(bars.q_full, 0) && mbar_wait(bars.k_full, 0);
-            if (ok) {
-                tc_fence_after();
-                for (int g = 0; g < nq; ++g) issue_qk(g, 0);
-            }
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int st = j % C::NSV;
-                const bool tail = (j == n_tiles - 1) && last_valid < C::BN;
-                uint64_t *bv = tail ? bars.v_tail : bars.v_full + st;
-                const uint32_t pv = tail ? 0u : (j / C::NSV) & 1;
-                const int jn = j + 1;
-                for (int g = 0; ok && g < nq; ++g) {
-                    // P V_j needs only V_j and this tile's P; Q K_{j+1}^T
-                    // waits for K_{j+1} after it, so a late K load does not
-                    // hold back the P*V that is ready
-                    if (!mbar_wait(bv, pv) || !mbar_wait(bars.p_ready + g, j & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_pv(g, j);
-                    if (jn < n_tiles) {
-                        if (g == 0 && !mbar_wait(bars.k_full + jn % C::NSK, (jn / C::NSK) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        issue_qk(g, jn);
-                    }
-                }
-            }
-            if (!ok) abort_cta();
-            mma_commit(bars.drain);
-            mbar_wait(bars.drain, 0);
-        }
-        __syncwarp();
-    } else if (warp >= kFirstSoftmaxWarp) {
-        // ------------------------------------------------------- softmax
-        regs_inc<kRegsSoftmax>();
-        const int grp = (warp - kFirstSoftmaxWarp) >> 2, wq = warp & 3;   // grp = query tile
-        const int r = wq * 32 + lane;
-        const int rg0 = row0 + grp * C::BM;                 // first row of this query tile
-        const bool warp_active = grp < nq && rg0 + wq * 32 < p.M;
-        const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t t_s = tmem + lane_addr + C::COL_S + grp * 128;
-        const uint32_t t_o = tmem + lane_addr + C::COL_O + grp * D;
-        const float c2 = p.scale_log2;
-        bool ok = true;
-        float m_run = -INFINITY;
-        uint64_t l_exact = 0, l_round = 0;
-        if (grp < nq) {
-            for (int j = 0; j < n_tiles; ++j) {
-                if (ok && !warp_wait(bars.s_full + grp, j & 1)) { ok = false; abort_cta(); }
-                tc_fence_after();
-                if (ok && warp_active) {
-                    const int n_valid = (j == n_tiles - 1) ? last_valid : C::BN;
-                    uint32_t r0[32], r1[32], r2[32], r3[32];
-                    tmem_ld32(t_s + 0, r0);
-                    tmem_ld32(t_s + 32, r1);
-                    tmem_ld32(t_s + 64, r2);
-                    tmem_ld32(t_s + 96, r3);
-                    tmem_wait_ld();
-                    if (n_valid < C::BN) {
-                        const uint32_t ninf = __float_as_uint(-INFINITY);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            r0[i] = (i < n_valid) ? r0[i] : ninf;
-                            r1[i] = (32 + i < n_valid) ? r1[i] : ninf;
-                            r2[i] = (64 + i < n_valid) ? r2[i] : ninf;
-                            r3[i] = (96 + i < n_valid) ? r3[i] : ninf;
-                        }
-                    }
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        m4[0] = max3(m4[0], __uint_as_float(r0[i]), __uint_as_float(r0[i + 1]));
-                        m4[1] = max3(m4[1], __uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
-                        m4[2] = max3(m4[2], __uint_as_float(r2[i]), __uint_as_float(r2[i + 1]));
-                        m4[3] = max3(m4[3], __uint_as_float(r3[i]), __uint_as_float(r3[i + 1]));
-                    }
-                    const float mt = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
-                    const float m_new = fmaxf(m_run, mt * c2);
-                    bool resc = false;
-                    float alpha = 1.f;
-                    if (m_new > m_run + 8.f) {                   // lazy update
-                        alpha = ex2(m_run - m_new);              // 0 on the first tile
-                        const uint64_t aa = f2(alpha, alpha);
-                        l_exact = fma2(l_exact, aa, 0ull);
-                        l_round = fma2(l_round, aa, 0ull);
-                        resc = j > 0;
-                        m_run = m_new;
-                    }
-                    const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-                    const uint64_t cc = f2(c2, c2), nm = f2(-mu, -mu);
-                    auto exps = [&](const uint32_t (&sc)[32], int col) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const uint64_t x2 = fma2(f2(__uint_as_float(sc[2 * k]), __uint_as_float(sc[2 * k + 1])),
-                                                     cc, nm);
-                            float p0, p1;
-                            if ((k & 3) == 3) {   // one pair in four on the FMA pipe
-                                const float2 e = exp2_poly2(x2);
-                                p0 = e.x;
-                                p1 = e.y;
-                            } else {
-                                const float2 x = unf2(x2);
-                                p0 = ex2(x.x);
-                                p1 = ex2(x.y);
-                            }
-                            pk[k] = pack_bf16x2(p0, p1);
-                            l_exact = add2(l_exact, f2(p0, p1));
-                            l_round = add2(l_round, f2(bf16_lo(pk[k]), bf16_hi(pk[k])));
-                        }
-                        tmem_st16(t_s + col, pk);
-                    };
-                    exps(r0, 0);
-                    exps(r1, 16);
-                    exps(r2, 32);
-                    exps(r3, 48);
-                    if (__any_sync(0xffffffffu, resc)) {
-                        // S of tile j was committed after P V_{j-1} of this query
-                        // tile was issued, so O[grp] is complete here
-                        const float a = resc ? alpha : 1.f;
-#pragma unroll 1
-                        for (int c = 0; c < D; c += 32) {
-                            uint32_t ro[32];
-                            tmem_ld32(t_o + c, ro);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * a);
-                            tmem_st32(t_o + c, ro);
-                        }
-                    }
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars.p_ready + grp);
-            }
-
-            // -------------------------------------------------- epilogue
-            if (ok && !warp_wait(bars.o_final, 0)) { ok = false; abort_cta(); }
-            tc_fence_after();
-            const bool failed = named_bar_or(1 + grp, 128, !ok || *s_abort);
-            const float2 le = unf2(l_exact), lr = unf2(l_round);
-            const float l_ex = le.x + le.y, l_rd = lr.x + lr.y;
-            if (!failed) {
-                // normalised rows into the staging area (16-byte chunks of a
-                // row XOR-swizzled by row % 8), then a coalesced copy-out
-                float *stage = reinterpret_cast<float *>(smem + (grp == 0 ? C::OFF_K : C::OFF_V));
-                const float inv = 1.f / l_rd;
-                if (warp_active) {
-#pragma unroll 1
-                    for (int c = 0; c < D; c += 32) {
-                        uint32_t x0[32];
-                        tmem_ld32(t_o + c, x0);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
-                            float4 v;
-                            v.x = __uint_as_float(x0[i + 0]) * inv;
-                            v.y = __uint_as_float(x0[i + 1]) * inv;
-                            v.z = __uint_as_float(x0[i + 2]) * inv;
-                            v.w = __uint_as_float(x0[i + 3]) * inv;
-                            const int q = (c + i) >> 2;
-                            *reinterpret_cast<float4 *>(stage + r * D + ((q ^ (r & 7)) << 2)) = v;
-                        }
-                    }
-                }
-                named_bar_sync(1 + grp, 128);
-                constexpr int CH = D / 4;
-                constexpr int RPI = 32 / CH;
-#pragma unroll 1
-                for (int base = wq * RPI; base < C::BM; base += 4 * RPI) {
-                    const int R = base + lane / CH, q = lane % CH;
-                    if (rg0 + R < p.M) {
-                        const float4 v = *reinterpret_cast<const float4 *>(stage + R * D + ((q ^ (R & 7)) << 2));
-                        *reinterpret_cast<float4 *>(p.o_part + ((grow0 + grp * C::BM + R) * p.S + split) * D + q * 4) = v;
-                    }
-                }
-            }
-            if (warp_active && rg0 + r < p.M)
-                p.lse_part[(grow0 + grp * C::BM + r) * p.S + split] = failed ? nan : (m_run + lg2(l_ex)) * kLn2;
-        }
-    } else {
-        regs_dec<kRegsOther>();   // warp 3: only completes the warpgroup
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        tc_fence_after();
-        tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-}
-
-template <int D>
-cudaError_t launch_pair(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                        const CUtensorMap &tm_v, cudaStream_t stream) {
-    using C = PairCfg<D>;
-    constexpr int kMaxDev = 64;
-    static bool attr_set[kMaxDev] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(prefix_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_ALLOC);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((p.M + 2 * C::BM - 1) / (2 * C::BM), p.S, p.B * p.Hkv);
-    cfg.blockDim = dim3(kThreadsTc);
-    cfg.dynamicSmemBytes = C::SMEM_ALLOC;
-    cfg.stream = stream;
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefix_pair_kernel<D>, tm_q, tm_k, tm_v, p);
-}
-
 template <int D, bool PAGED, bool WINDOW>
 cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                       const CUtensorMap &tm_v, cudaStream_t stream) {
@@ -1235,9 +773,6 @@ cudaError_t launch_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUte
 cudaError_t launch_prefix_tc(const PrefixParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                              const CUtensorMap &tm_v, cudaStream_t stream) {
     const bool paged = p.block_table != nullptr;
-    if (p.pair && !paged && p.window == 0 && p.M > 128)
-        return p.D == 128 ? launch_pair<128>(p, tm_q, tm_k, tm_v, stream)
-                          : launch_pair<64>(p, tm_q, tm_k, tm_v, stream);
     if (p.window > 0)
         return p.D == 128 ? launch_tc<128, false, true>(p, tm_q, tm_k, tm_v, stream)
                           : launch_tc<64, false, true>(p, tm_q, tm_k, tm_v, stream);

@@ -37,7 +37,6 @@ ERR_BAD_PATH = -21
 
 PREFIX_TCGEN05 = 0
 PREFIX_SIMT = 1
-PREFIX_TCGEN05_PAIR = 2     # tcgen05, two query tiles per CTA when G*T > 128 (slower)
 T_MAX = 256
 
 EXPORTED = [
@@ -46,7 +45,7 @@ EXPORTED = [
     "longspec_hta_workspace_bytes", "longspec_hta_workspace_init", "longspec_hta_verify",
     "longspec_hta_verify_ex", "longspec_hta_host_arena_bytes", "longspec_hta_verify_host",
     "longspec_hta_tree_mask", "longspec_hta_tree_partial", "longspec_hta_prefix_partial",
-    "longspec_hta_get_status", "longspec_hta_verify_noalloc",
+    "longspec_hta_get_status", "longspec_hta_verify_noalloc", "longspec_hta_noalloc_chunking",
     "longspec_hta_selftest_wait_timeout", "longspec_hta_prefix_attention",
     "longspec_hta_verify_paged", "longspec_hta_prefix_attention_paged",
     "longspec_hta_accept_workspace_bytes", "longspec_hta_accept_greedy",
@@ -120,6 +119,7 @@ def load():
             lib.longspec_hta_get_status.argtypes = [vp, vp]
             lib.longspec_hta_selftest_wait_timeout.argtypes = [vp, vp]
             lib.longspec_hta_chunking.argtypes = [pd, ci, ctypes.POINTER(ci), ctypes.POINTER(ci)]
+            lib.longspec_hta_noalloc_chunking.argtypes = [pd, ci, ctypes.POINTER(ci), ctypes.POINTER(ci)]
             lib.longspec_hta_accept_workspace_bytes.argtypes = [ci, ci, ci]
             lib.longspec_hta_accept_workspace_bytes.restype = sz
             lib.longspec_hta_accept_greedy.argtypes = [ci, ci, ci] + [vp] * 6 + [vp, sz, vp]
@@ -175,6 +175,15 @@ def chunking(dims: Dims, num_splits: int = 0):
     S, C = ctypes.c_int(0), ctypes.c_int(0)
     _check(load().longspec_hta_chunking(ctypes.byref(dims), int(num_splits), ctypes.byref(S),
                                         ctypes.byref(C)))
+    return S.value, C.value
+
+
+def noalloc_chunking(dims: Dims, num_sms: int):
+    """(S, chunk_keys) longspec_hta_verify_noalloc uses on a GPU with
+    num_sms SMs (host only)."""
+    S, C = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().longspec_hta_noalloc_chunking(ctypes.byref(dims), int(num_sms), ctypes.byref(S),
+                                                ctypes.byref(C)))
     return S.value, C.value
 
 
