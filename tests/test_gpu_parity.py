@@ -250,6 +250,27 @@ def test_deterministic_bits():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("name", ["llama3-8b-32k", "qwq-32b-32k-peaked"])
+def test_deterministic_bits_full_size(name):
+    """Repeated calls at full size (43 key tiles per CTA, a 16-row remainder
+    tile) give the same bits: a pipeline race between the warps of a CTA
+    would show here first."""
+    w = WORKLOADS[name]
+    dev = H.make_inputs(w)
+    ws = hta.new_workspace(hta.dims_of(dev["q"], dev["k_prefix"], w.scale))
+    ref = None
+    for _ in range(3):
+        o, l = hta.verify(dev["q"], dev["k_prefix"], dev["v_prefix"], dev["prefix_len"],
+                          dev["k_tree"], dev["v_tree"], dev["parent"], workspace=ws)
+        assert hta.get_status(ws) == hta.OK
+        if ref is None:
+            ref = (o.clone(), l.clone())
+        else:
+            assert torch.equal(o, ref[0]) and torch.equal(l, ref[1])
+    del dev
+    torch.cuda.empty_cache()
+
+
 def test_host_buffer_entry_point_matches_device_call():
     w = SMALL["vicuna-like-ragged"]
     cpu = {k: v.pin_memory() for k, v in w.generate().items()}
