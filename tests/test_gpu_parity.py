@@ -106,6 +106,25 @@ def test_tree_partial_matches_oracle(name):
     H.assert_parity(o, l, ro, rl, f"tree/{name}")
 
 
+@pytest.mark.parametrize("name", ["llama-like-L1000", "max-tree-256", "deep-chain-256", "tiny",
+                                  "d64-random-tree"])
+def test_verify_with_empty_prefix_is_the_tree_partial(name):
+    """With L_b = 0 for every sequence a verification call sees its tree keys
+    only, so its out / lse are the oracle's tree-only pass (lse at 1e-3):
+    the tree pass of the full call, trees of up to 256 nodes and 256-deep
+    chains included, with every prefix chunk empty."""
+    w = SMALL[name]
+    cpu = w.generate()
+    cpu["prefix_len"].zero_()
+    ro, rl = H.oracle_problem(cpu, w.scale).tree_partial()
+    dev = H.to_device(cpu)
+    ws = hta.new_workspace(hta.dims_of(dev["q"], dev["k_prefix"], w.scale))
+    out, lse = hta.verify(dev["q"], dev["k_prefix"], dev["v_prefix"], dev["prefix_len"],
+                          dev["k_tree"], dev["v_tree"], dev["parent"], workspace=ws, scale=w.scale)
+    assert hta.get_status(ws) == hta.OK
+    H.assert_parity(out, lse, ro, rl, f"empty prefix = tree partial/{name}")
+
+
 def _trees():
     out = []
     for name in ("llama3-8b-32k", "vicuna-7b-b8", "tiny", "ultra-256k-chain5"):
