@@ -69,12 +69,22 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
 #pragma unroll
             for (int u = 0; u < KB; ++u) {
                 const int j = idx[u] < 0 ? idx[0] : idx[u];
+                // a key row is D contiguous bf16: one vector load per lane,
+                // the warp reading the row as one coalesced 2*D-byte access
                 const __nv_bfloat16 *kr = p.k_tree + (kv_base + j) * D + lane * DPL;
                 const __nv_bfloat16 *vr = p.v_tree + (kv_base + j) * D + lane * DPL;
-#pragma unroll
-                for (int i = 0; i < DPL; ++i) {
-                    kf[u][i] = __bfloat162float(kr[i]);
-                    vf[u][i] = __bfloat162float(vr[i]);
+                if constexpr (DPL == 4) {
+                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr);
+                    const uint2 vv = *reinterpret_cast<const uint2 *>(vr);
+                    kf[u][0] = bf16_lo(kk.x); kf[u][1] = bf16_hi(kk.x);
+                    kf[u][2] = bf16_lo(kk.y); kf[u][3] = bf16_hi(kk.y);
+                    vf[u][0] = bf16_lo(vv.x); vf[u][1] = bf16_hi(vv.x);
+                    vf[u][2] = bf16_lo(vv.y); vf[u][3] = bf16_hi(vv.y);
+                } else {
+                    const uint32_t kk = *reinterpret_cast<const uint32_t *>(kr);
+                    const uint32_t vv = *reinterpret_cast<const uint32_t *>(vr);
+                    kf[u][0] = bf16_lo(kk); kf[u][1] = bf16_hi(kk);
+                    vf[u][0] = bf16_lo(vv); vf[u][1] = bf16_hi(vv);
                 }
             }
             float x[KB];
@@ -122,12 +132,14 @@ __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWo
         return;
     }
 
-    // merge: the tree partial (m, l, acc; log2 units) with S prefix partials
+    // merge: the tree partial (m, l, acc; log2 units) with S prefix partials.
+    // prefix_len is an input of the call, like q and the tree K/V above:
+    // read before the wait, so the partials' loads follow it directly.
+    const int L = p.prefix_len[b];
     grid_dependency_wait();   // the prefix kernel's partials are complete and visible
     // The next kernel on the stream (the next call's prefix pass) may be
     // scheduled now: it waits for this grid before it reads anything.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int L = p.prefix_len[b];
     const bool bad_len = L < 0 || (p.window == 0 && L > p.L_cap);
     if (bad_len && lane == 0 && rr == 0) raise_status(p.status, kStatusPrefixLenRange);
     float out_v[DPL];
@@ -309,14 +321,32 @@ __device__ __forceinline__ void arg_take(ArgBest &b, float v, int i) {
     if (v > b.v || (v == b.v && i < b.i)) { b.v = v; b.i = i; }
 }
 
-__device__ __forceinline__ void arg_take8(ArgBest &b, uint4 u, int i0) {
-    arg_take(b, bf16_lo(u.x), i0 + 0); arg_take(b, bf16_hi(u.x), i0 + 1);
-    arg_take(b, bf16_lo(u.y), i0 + 2); arg_take(b, bf16_hi(u.y), i0 + 3);
-    arg_take(b, bf16_lo(u.z), i0 + 4); arg_take(b, bf16_hi(u.z), i0 + 5);
-    arg_take(b, bf16_lo(u.w), i0 + 6); arg_take(b, bf16_hi(u.w), i0 + 7);
+constexpr int kArgThreads = 256;
+
+// The larger of each bf16 pair (max.bf16x2: a NaN loses to a number).
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
-constexpr int kArgThreads = 256;
+// Largest of the 8 bf16 values of a 16-byte chunk, as fp32 (NaN only if all
+// 8 are NaN).
+__device__ __forceinline__ float chunk_max8(uint4 u) {
+    const uint32_t m = max_bf16x2(max_bf16x2(u.x, u.y), max_bf16x2(u.z, u.w));
+    return fmaxf(bf16_lo(m), bf16_hi(m));
+}
+
+// Position (0..7) of the first of the 8 values of `u` equal to `v`
+// (8 if none).
+__device__ __forceinline__ int first_equal8(uint4 u, float v) {
+    int e = 8;
+    e = (bf16_hi(u.w) == v) ? 7 : e; e = (bf16_lo(u.w) == v) ? 6 : e;
+    e = (bf16_hi(u.z) == v) ? 5 : e; e = (bf16_lo(u.z) == v) ? 4 : e;
+    e = (bf16_hi(u.y) == v) ? 3 : e; e = (bf16_lo(u.y) == v) ? 2 : e;
+    e = (bf16_hi(u.x) == v) ? 1 : e; e = (bf16_lo(u.x) == v) ? 0 : e;
+    return e;
+}
 
 }  // namespace
 
@@ -336,15 +366,36 @@ argmax_slices_kernel(const __nv_bfloat16 *logits, int V, int slice, float *part_
     if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
         const uint4 *xv = reinterpret_cast<const uint4 *>(x);
         const int c_lo = lo / 8, c_hi = hi / 8;            // whole 8-element chunks
-        // up to eight 16-byte loads in flight per thread, then their compares
+        // Up to eight 16-byte loads in flight per thread, then: the max of
+        // each chunk (packed bf16 max), the batch max, and only where it
+        // beats the best so far the first chunk and element holding it.  A
+        // batch's indices grow with k and lie above every earlier batch's,
+        // so the first match is the smallest index.  A batch holding only
+        // NaN and -inf (all count as -inf) offers its first element.
         for (int c = c_lo + threadIdx.x; c < c_hi; c += 8 * kArgThreads) {
             uint4 u[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 u[k] = c + k * kArgThreads < c_hi ? __ldcs(xv + c + k * kArgThreads) : make_uint4(0u, 0u, 0u, 0u);
+            float cm[8];
+            float tm = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                if (c + k * kArgThreads < c_hi) arg_take8(b, u[k], 8 * (c + k * kArgThreads));
+            for (int k = 0; k < 8; ++k) {
+                cm[k] = c + k * kArgThreads < c_hi ? chunk_max8(u[k]) : -INFINITY;
+                tm = fmaxf(tm, cm[k]);   // a NaN chunk max (all NaN) loses
+            }
+            if (tm > b.v) {
+                int kk = 0;
+#pragma unroll
+                for (int k = 7; k >= 0; --k) kk = (cm[k] == tm) ? k : kk;
+                uint4 w = u[0];
+#pragma unroll
+                for (int k = 1; k < 8; ++k) w = (k == kk) ? u[k] : w;
+                b.v = tm;
+                b.i = 8 * (c + kk * kArgThreads) + first_equal8(w, tm);
+            } else if (b.i == INT_MAX) {
+                b.i = 8 * c;   // nothing above -inf yet: this batch's first element
+            }
         }
         for (int i = c_hi * 8 + threadIdx.x; i < hi; i += kArgThreads) arg_take(b, __bfloat162float(x[i]), i);
     } else {
