@@ -67,17 +67,33 @@ def workload_config(w, S, n_sets):
             if n_sets > 1 else "K/V bytes per call > 2x L2"}
 
 
-def profiled_traffic(workload_name, kernel_file="tree_masked_verification_b200/csrc/prefix_tc.cu"):
+PREFIX_KERNEL_SOURCES = ("tree_masked_verification_b200/csrc/prefix_tc.cu",
+                         "tree_masked_verification_b200/csrc/hta_kernels.h",
+                         "tree_masked_verification_b200/csrc/hta_common.cuh")
+
+
+def prefix_source_sha():
+    """First 16 hex digits of the SHA-256 of the prefix kernel's sources
+    (the kernel file and the two headers it compiles with, concatenated)."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in PREFIX_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload_name):
     """DRAM bytes per launch of the prefix kernel from the committed ncu
     summary, if that summary was taken on this workload with the current
-    kernel source (else None)."""
-    import hashlib
+    kernel sources and the default build (else None)."""
+    if os.environ.get("LONGSPEC_HTA_LIB"):
+        return None          # another build than the one profiled
     path = os.path.join(ROOT, "profiles", f"prefix_tc_kernel_{workload_name}.json")
     try:
         with open(path) as f:
             prof = json.load(f)
-        with open(os.path.join(ROOT, kernel_file), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        sha = prefix_source_sha()
     except (OSError, ValueError):
         return None
     if prof.get("source_sha256_16") != sha:
@@ -572,6 +588,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 2 * args.steps,
         "timing": "value: CUDA events around the K back-to-back calls; roofline: a second pass "
                   "of the same calls with events around each prefix launch",
+        "build": {"library": os.path.basename(hta.library_path()), **hta.build_info()},
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -134,6 +134,13 @@ typedef struct {
 /* ABI version of the loaded library (LONGSPEC_HTA_ABI_VERSION). */
 LONGSPEC_HTA_API int longspec_hta_abi_version(void);
 
+/* Build-time tuning of the loaded library, as "key=value" pairs separated
+ * by spaces: kv_stages_d128 (K/V ring depth of the tcgen05 prefix kernel at
+ * D = 128) and exp2_poly_every (one exp2 pair in this many evaluated on the
+ * FMA pipe, 0 = none).  A static string owned by the library; never NULL.
+ * Lets a benchmark record which build it timed. */
+LONGSPEC_HTA_API const char *longspec_hta_build_info(void);
+
 /* Text of a status code; never NULL. */
 LONGSPEC_HTA_API const char *longspec_hta_strerror(int code);
 

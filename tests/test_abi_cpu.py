@@ -275,3 +275,10 @@ def test_noalloc_chunking_rejects_what_one_split_cannot_hold(lib):
     rc = lib.longspec_hta_noalloc_chunking(ctypes.byref(d), 148, ctypes.byref(S), ctypes.byref(C))
     assert rc == hta.ERR_WORKSPACE_TOO_SMALL
     assert lib.longspec_hta_noalloc_chunking(ctypes.byref(_dims()), 0, None, None) == hta.ERR_INVALID_OPTION
+
+
+def test_build_info_reports_the_tuning_knobs(lib):
+    """The in-tree build carries the default knobs of csrc/hta_kernels.h."""
+    lib.longspec_hta_build_info.restype = ctypes.c_char_p
+    text = lib.longspec_hta_build_info().decode()
+    assert dict(kv.split("=") for kv in text.split()) == {"kv_stages_d128": "3", "exp2_poly_every": "4"}

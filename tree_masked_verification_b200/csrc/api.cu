@@ -252,6 +252,12 @@ extern "C" {
 
 int longspec_hta_abi_version(void) { return LONGSPEC_HTA_ABI_VERSION; }
 
+#define HTA_STR2(x) #x
+#define HTA_STR(x) HTA_STR2(x)
+const char *longspec_hta_build_info(void) {
+    return "kv_stages_d128=" HTA_STR(HTA_KV_STAGES_D128) " exp2_poly_every=" HTA_STR(HTA_EXP2_POLY_EVERY);
+}
+
 const char *longspec_hta_strerror(int code) {
     switch (code) {
     case LONGSPEC_HTA_OK: return "ok";

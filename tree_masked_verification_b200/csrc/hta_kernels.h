@@ -9,6 +9,23 @@
 
 #include "hta_common.cuh"
 
+// Build-time tuning knobs of the tcgen05 prefix kernel (defaults = the
+// measured best on B200; set with -D at build time, reported by
+// longspec_hta_build_info):
+//   HTA_KV_STAGES_D128   depth of the K and V rings at D = 128 (2 or 3; four
+//                        stages of 32 KB each do not fit beside Q)
+//   HTA_EXP2_POLY_EVERY  one exp2 pair in this many on the FMA pipe (0: all
+//                        on the exp2 unit; 2, 4, 8 or 16)
+#ifndef HTA_KV_STAGES_D128
+#define HTA_KV_STAGES_D128 3
+#endif
+#ifndef HTA_EXP2_POLY_EVERY
+#define HTA_EXP2_POLY_EVERY 4
+#endif
+static_assert(HTA_KV_STAGES_D128 == 2 || HTA_KV_STAGES_D128 == 3, "K/V ring depth at D = 128");
+static_assert(HTA_EXP2_POLY_EVERY == 0 || HTA_EXP2_POLY_EVERY == 2 || HTA_EXP2_POLY_EVERY == 4 ||
+              HTA_EXP2_POLY_EVERY == 8 || HTA_EXP2_POLY_EVERY == 16, "exp2 share on the FMA pipe");
+
 namespace hta {
 
 constexpr int kTreeRowsPerCta = 8;    // one warp per packed row

@@ -49,7 +49,7 @@ template <int D>
 struct TcCfg {
     static constexpr int BM = 128;
     static constexpr int BN = kKeyTile;                     // 128 keys per tile
-    static constexpr int NS = (D == 128) ? 3 : 4;           // K and V ring depth
+    static constexpr int NS = (D == 128) ? HTA_KV_STAGES_D128 : 4;   // K and V ring depth
     static constexpr int HALVES = D / 64;                   // 64-column swizzle boxes
     static constexpr int BOX_BYTES = 128 * 64 * 2;          // one 128-row x 64-col box
     static constexpr int Q_BYTES = BM * D * 2;
@@ -614,7 +614,8 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const uint64_t x2 = fma2(f2(__uint_as_float(sc[2 * k]), __uint_as_float(sc[2 * k + 1])),
                                                  cc, nm);
                         float p0, p1;
-                        if ((k & 3) == 3) {   // one pair in four on the FMA pipe
+                        constexpr int kEvery = HTA_EXP2_POLY_EVERY;   // default: one pair in four
+                        if (kEvery > 0 && k % kEvery == kEvery - 1) {   // this pair on the FMA pipe
                             const float2 e = exp2_poly2(x2);
                             p0 = e.x;
                             p1 = e.y;

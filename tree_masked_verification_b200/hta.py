@@ -14,7 +14,10 @@ import threading
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblongspec_hta.so")
+# The in-tree build; LONGSPEC_HTA_LIB names another build of the same
+# library instead (a build with other tuning knobs, for A/B timing).
+_LIB_PATH = os.environ.get("LONGSPEC_HTA_LIB") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "liblongspec_hta.so")
 _lock = threading.Lock()
 _lib = None
 
@@ -40,7 +43,7 @@ PREFIX_SIMT = 1
 T_MAX = 256
 
 EXPORTED = [
-    "longspec_hta_abi_version", "longspec_hta_strerror", "longspec_hta_default_splits",
+    "longspec_hta_abi_version", "longspec_hta_build_info", "longspec_hta_strerror", "longspec_hta_default_splits",
     "longspec_hta_chunking",
     "longspec_hta_workspace_bytes", "longspec_hta_workspace_init", "longspec_hta_verify",
     "longspec_hta_verify_ex", "longspec_hta_host_arena_bytes", "longspec_hta_verify_host",
@@ -97,6 +100,7 @@ def load():
             vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             pd = ctypes.POINTER(Dims)
             lib.longspec_hta_abi_version.restype = ci
+            lib.longspec_hta_build_info.restype = ctypes.c_char_p
             lib.longspec_hta_strerror.argtypes = [ci]
             lib.longspec_hta_strerror.restype = ctypes.c_char_p
             lib.longspec_hta_default_splits.argtypes = [pd]
@@ -516,6 +520,13 @@ def selftest_wait_timeout(workspace: torch.Tensor, stream=None) -> int:
     one bounded in-kernel wait that nothing completes (about 2 s); a later
     get_status() returns ERR_PIPELINE_TIMEOUT."""
     return int(load().longspec_hta_selftest_wait_timeout(_ptr(workspace), _stream(stream)))
+
+
+def build_info() -> dict:
+    """The loaded library's build-time tuning knobs, e.g.
+    {"kv_stages_d128": 3, "exp2_poly_every": 4}."""
+    text = load().longspec_hta_build_info().decode()
+    return {k: int(v) for k, v in (kv.split("=") for kv in text.split())}
 
 
 def get_status(workspace: torch.Tensor, stream=None) -> int:
