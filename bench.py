@@ -546,7 +546,7 @@ def run_ours(args, world, rank, local):
         call(i)
     host_us = (time.perf_counter() - h0) / n_host * 1e6
     torch.cuda.synchronize()
-    c_abi_us = c_abi_host_us(w, sets[0], out, lse, ws, dims, stream, n_host)
+    c_abi_us = c_abi_host_us(w, sets[0], out, lse, ws, dims, stream, n_host, args.num_splits)
     torch.cuda.synchronize()
 
     ms_per_step = elapsed_ms / args.steps
@@ -762,8 +762,8 @@ def run_accept(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
-def c_abi_host_us(w, s, out, lse, ws, dims, stream, n):
-    """Host time of one longspec_hta_verify call on its own: the C entry
+def c_abi_host_us(w, s, out, lse, ws, dims, stream, n, num_splits=0):
+    """Host time of one longspec_hta_verify_ex call on its own: the C entry
     point called in a loop with its arguments converted once, so the figure
     holds the library's checks, tensor-map lookups and launches but not the
     Python binding's marshalling (the GPU runs behind).  None for calls other
@@ -771,13 +771,14 @@ def c_abi_host_us(w, s, out, lse, ws, dims, stream, n):
     import ctypes
     if w.kind != "verify" or w.block_size:
         return None
-    fn = hta.load().longspec_hta_verify
+    fn = hta.load().longspec_hta_verify_ex
+    opts = hta.Options(num_splits, hta.PREFIX_TCGEN05, None, None)
     args = (ctypes.byref(dims), s["q"].data_ptr(), s["k_prefix"].data_ptr(), s["v_prefix"].data_ptr(),
             s["prefix_len"].data_ptr(), s["k_tree"].data_ptr(), s["v_tree"].data_ptr(),
             s["parent"].data_ptr(), out.data_ptr(), lse.data_ptr(), ws.data_ptr(),
-            ws.numel(), stream.cuda_stream)
+            ws.numel(), ctypes.byref(opts), stream.cuda_stream)
     if fn(*args) != hta.OK:
-        raise RuntimeError("longspec_hta_verify failed")
+        raise RuntimeError("longspec_hta_verify_ex failed")
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for _ in range(n):
