@@ -189,6 +189,34 @@ __device__ __forceinline__ float2 exp2_poly2(uint64_t x2) {
     return o;
 }
 
+// L2 eviction policies (createpolicy) and the hinted TMA load / store
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                                                 int x, int y, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)),
+          "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void st_v4_hint(float *dst, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;"
+                 ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_f32_hint(float *dst, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(dst), "f"(v), "l"(pol) : "memory");
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -271,6 +299,10 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         raise_status(p.status, kStatusPipelineTimeout);
     };
     const int kv_row0 = bk * p.L_cap + key_begin;
+    // K/V read by one row tile only (G*T <= 128): each line is used once,
+    // so it is marked first to leave L2, which keeps the split partials
+    // (marked last) there until the merge reads them
+    const bool stream_once = p.m_tiles == 1;
     // Producer of a K or V ring from a paged cache, run by the whole warp.
     // A 128-key tile is read with one block_size-row box per block and
     // 64-column half, each landing at the block's rows of the swizzled stage
@@ -337,6 +369,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (warp == kProducerKWarp) {
         // -------------------------------------------------------- TMA: Q, K
         regs_dec<kRegsOther>();
+        const uint64_t kv_pol = l2_policy_evict_first();
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -371,8 +404,12 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint8_t *sk = smem + C::OFF_K + st * C::KV_BYTES;
                 mbar_arrive_expect_tx(bars.k_full + st, C::KV_BYTES);
 #pragma unroll
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_2d(sk + h * C::BOX_BYTES, &tm_k, bars.k_full + st, h * 64, kv_row0 + j * C::BN);
+                for (int h = 0; h < C::HALVES; ++h) {
+                    if (stream_once)
+                        tma_load_2d_hint(sk + h * C::BOX_BYTES, &tm_k, bars.k_full + st, h * 64, kv_row0 + j * C::BN, kv_pol);
+                    else
+                        tma_load_2d(sk + h * C::BOX_BYTES, &tm_k, bars.k_full + st, h * 64, kv_row0 + j * C::BN);
+                }
                 issued = j + 1;
             }
             if (*s_abort) {
@@ -386,6 +423,7 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     } else if (warp == kProducerVWarp) {
         // ----------------------------------------------------------- TMA: V
         regs_dec<kRegsOther>();
+        const uint64_t kv_pol = l2_policy_evict_first();
         if (lane == 0) tma_prefetch_desc(&tm_v);
         if constexpr (PAGED) {
             const int issued = paged_ring(smem + C::OFF_V, &tm_v, bars.v_full, bars.v_empty);
@@ -410,8 +448,12 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint8_t *sv = smem + C::OFF_V + st * C::KV_BYTES;
                 mbar_arrive_expect_tx(bars.v_full + st, C::KV_BYTES);
 #pragma unroll
-                for (int h = 0; h < C::HALVES; ++h)
-                    tma_load_2d(sv + h * C::BOX_BYTES, &tm_v, bars.v_full + st, h * 64, kv_row0 + j * C::BN);
+                for (int h = 0; h < C::HALVES; ++h) {
+                    if (stream_once)
+                        tma_load_2d_hint(sv + h * C::BOX_BYTES, &tm_v, bars.v_full + st, h * 64, kv_row0 + j * C::BN, kv_pol);
+                    else
+                        tma_load_2d(sv + h * C::BOX_BYTES, &tm_v, bars.v_full + st, h * 64, kv_row0 + j * C::BN);
+                }
                 issued = j + 1;
             }
             if (*s_abort) {
@@ -657,6 +699,9 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
 
         // ------------------------------------------------------ epilogue
+        // the partials are read back by the merge right after this grid:
+        // kept in L2 ahead of the K/V lines
+        const uint64_t part_pol = l2_policy_evict_last();
         if (ok && !warp_wait(bars.o_final, 0)) { ok = false; abort_cta(); }
         tc_fence_after();
         // merge the two groups' online softmaxes row by row (the lse merge
@@ -720,12 +765,12 @@ prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int R = base + lane / CH, q = lane % CH;
                 if (row0 + R < p.M) {
                     const float4 v = *reinterpret_cast<const float4 *>(stage + R * D + ((q ^ (R & 7)) << 2));
-                    *reinterpret_cast<float4 *>(p.o_part + ((grow0 + R) * p.S + split) * D + q * 4) = v;
+                    st_v4_hint(p.o_part + ((grow0 + R) * p.S + split) * D + q * 4, v, part_pol);
                 }
             }
         }
         if (grp == 0 && warp_active && rr < p.M)
-            p.lse_part[(grow0 + r) * p.S + split] = failed ? nan : (m + lg2(l_ex)) * kLn2;
+            st_f32_hint(p.lse_part + (grow0 + r) * p.S + split, failed ? nan : (m + lg2(l_ex)) * kLn2, part_pol);
     }
 
     else {
