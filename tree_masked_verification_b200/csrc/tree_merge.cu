@@ -12,7 +12,7 @@
 //      jump[i] = jump[jump[i]]), so deep chains cost no more than bushy trees,
 //   3. runs, one warp per row, the online softmax over the visible tree keys
 //      only (the mask bits are walked, never the full T x T grid), fetching
-//      up to 8 visible keys' K and V rows at once,
+//      up to 4 visible keys' K and V rows at once,
 //   4. waits for the prefix kernel (programmatic dependent launch: steps 1-3
 //      overlap the prefix kernel's tail) and merges the tree partial with the
 //      S split-KV partials by log-sum-exp rescaling, writing out (bf16) and
@@ -35,7 +35,7 @@ template <int D>
 __device__ void tree_row(const TreeMergeParams &p, const uint32_t (*anc)[kMaskWords], int b,
                          int kvh, int rr, bool bad_parent) {
     constexpr int DPL = D / 32;   // values per lane
-    constexpr int KB = 8;         // visible keys fetched at once
+    constexpr int KB = 4;         // visible keys fetched at once
     const int lane = threadIdx.x % 32;
     const int G = p.Hq / p.Hkv, W = (p.T + 31) / 32;
     const float nan = __int_as_float(0x7fc00000);
@@ -272,7 +272,9 @@ __device__ bool build_tree_mask(const int32_t *parent_b, int T, int *s_jump,
     return bad;
 }
 
-__global__ void __launch_bounds__(kThreads)
+// At most 64 registers (four CTAs per SM): the kernel is latency-bound, so
+// more resident warps pay more than deeper batches of key loads.
+__global__ void __launch_bounds__(kThreads, 4)
 tree_merge_kernel(TreeMergeParams p) {
     __shared__ int s_jump[kTMax];
     __shared__ uint32_t s_anc[kTMax][kMaskWords];
