@@ -569,10 +569,13 @@ int longspec_hta_prefix_attention_paged(const longspec_hta_dims *dims, const voi
 // ---- greedy acceptance ------------------------------------------------------
 namespace {
 constexpr int kAcceptMaxSlices = 32;
-// slices per logits row: enough CTAs to keep every SM streaming
+// slices per logits row: about two CTAs per SM over the grid (measured on
+// B200 against one, four, eight and sixteen: fewer, longer slices lose the
+// parallelism of a short wave, more of them add CTAs whose ramp and
+// reduction outweigh their share of the stream)
 int accept_slices(int B, int T, int V, int num_sms) {
     const long long rows = 1LL * B * (T + 1);
-    long long want = (4LL * num_sms + rows - 1) / rows;
+    long long want = (2LL * num_sms + rows - 1) / rows;
     want = std::min<long long>(want, (V + 2047) / 2048);     // at least 2048 elements a slice
     return static_cast<int>(std::max<long long>(1, std::min<long long>(want, kAcceptMaxSlices)));
 }
